@@ -1,0 +1,8 @@
+"""CPU fp64 oracle (test infrastructure only; see mla_oracle's header)."""
+from .mla_oracle import (  # noqa: F401
+    cache_elements_per_token,
+    cache_rows,
+    decode_absorbed,
+    decode_expanded,
+    rope,
+)
