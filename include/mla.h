@@ -1,0 +1,186 @@
+/*
+ * mla.h -- C ABI of libmla.so: absorbed Multi-head Latent Attention (MLA)
+ * decode on NVIDIA B200 (sm_100a).
+ *
+ * The method (DeepSeek-V3 MLA, decode step, absorbed order):
+ *   - per token and layer the cache keeps only a latent c_KV (d_c = 512) and a
+ *     decoupled RoPE key k_R (d_r = 64), 576 numbers
+ *     (wq-win.github.io/llm/092-deepseekv3.html, section 二 "MLA：缓存压缩后的历史";
+ *      ailearn.mscapital.top/deepseek-v3.html, MLA paragraph after the
+ *      configuration table);
+ *   - each head's content query is folded through W_UK into latent space and
+ *     dotted with every cached c_KV; the RoPE score q_R . k_R is added
+ *     separately (092 page, section 二 "缓存压缩也可以做一个代数检查":
+ *      q^T (U c) = (U^T q)^T c; m.lsln.cn/news/222502 sections 2.2 and 2.3);
+ *   - softmax over the whole history, aggregate sum_j p_j c_KV,j in latent
+ *     space, then map through W_UV to the per-head output
+ *     (ailearn.mscapital.top/deepseek-v3.html, MLA "状态传导图" panel).
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers unless stated otherwise; the
+ *     caller owns every buffer, and the library keeps no pointer after a call
+ *     returns.  Tensors are dense and row-major in the layouts given below.
+ *   - dtype: MLA_DTYPE_BF16 (storage bf16, fp32 accumulation) or
+ *     MLA_DTYPE_F32.  Every tensor of one call has the call's dtype, except
+ *     positions / seqlens (int32) and the workspace (bytes).
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream) and never synchronise the host, except
+ *     mla_device_status().
+ *   - Return value: MLA_OK (0) or a negative MLA_ERR_* code.  On error nothing
+ *     was launched and mla_last_error() (thread-local) describes why.
+ *   - Values that live on the device (positions, seqlens) are checked by the
+ *     kernels: a bad value sets a bit in the library's device status word and
+ *     the affected rows are skipped (append) or written as zeros (decode);
+ *     mla_device_status() reports and clears the word.
+ *   - Pointers must be 16-byte aligned (MLA_ERR_ALIGN otherwise).
+ */
+#ifndef MLA_H_
+#define MLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* mla_stream_t; /* same type as cudaStream_t */
+
+enum {
+    MLA_OK = 0,
+    MLA_ERR_ARG = -1,         /* NULL pointer, negative size, bad enum */
+    MLA_ERR_SHAPE = -2,       /* dimensions outside what an entry point supports */
+    MLA_ERR_ALIGN = -3,       /* pointer or stride not 16-byte aligned */
+    MLA_ERR_CUDA = -4,        /* a CUDA runtime/driver call failed */
+    MLA_ERR_TIMEOUT = -5,     /* a device-side wait gave up (see mla_device_status) */
+    MLA_ERR_DEVICE = -6,      /* device status word non-zero (bad positions/seqlens) */
+    MLA_ERR_WORKSPACE = -7,   /* workspace NULL or smaller than mla_workspace_bytes() */
+    MLA_ERR_UNSUPPORTED = -8  /* a forced path cannot run this shape / device */
+};
+
+enum { MLA_DTYPE_BF16 = 0, MLA_DTYPE_F32 = 1 };
+
+/* Head geometry.  V3 values: H=128, d_c=512, d_r=64, d_n=128, d_v=128
+ * (ailearn.mscapital.top/deepseek-v3.html, configuration table, row "MLA").
+ * rope_base: RoPE frequency base (10000).  softmax_scale: 0 selects
+ * 1/sqrt(d_n + d_r). */
+typedef struct {
+    int32_t H, d_c, d_r, d_n, d_v;
+    int32_t dtype;
+    float rope_base;
+    float softmax_scale;
+} mla_dims_t;
+
+/* The compressed KV cache: B sequences x T_max rows; row t of sequence b
+ * starts at data + b*stride_b + t*stride_t (strides in ELEMENTS) and holds
+ * d_c latent values followed by d_r RoPE-key values already rotated at
+ * position t.  stride_t >= d_c + d_r; strides*elem_size multiples of 16. */
+typedef struct {
+    void* data;
+    int32_t B, T_max;
+    int64_t stride_b, stride_t;
+} mla_cache_t;
+
+/* Device status bits (mla_device_status). */
+enum {
+    MLA_STATUS_BAD_POS = 1,     /* append: pos[b] < 0 or pos[b] + n_tok > T_max */
+    MLA_STATUS_BAD_SEQLEN = 2,  /* decode: seqlens[b] < q_len or > T_max */
+    MLA_STATUS_TIMEOUT = 4      /* a bounded device-side wait expired */
+};
+
+/* ---------------------------------------------------------------- a1: append
+ * Write n_tok new tokens per sequence into the cache (092 page, section 二
+ * "MLA：缓存压缩后的历史": the cache keeps c_KV and the RoPE key).
+ *   c_kv   [B][n_tok][d_c]   latent of each new token
+ *   k_rope [B][n_tok][d_r]   UN-rotated RoPE key; rotated here at its position
+ *   pos    [B] int32         position of the first new token of sequence b
+ * Row pos[b]+i of sequence b becomes [c_kv[b][i] || RoPE(k_rope[b][i], pos[b]+i)].
+ * Rows with an out-of-range position are skipped and flag MLA_STATUS_BAD_POS. */
+int mla_append_cache(const mla_dims_t* dims, const void* c_kv, const void* k_rope,
+                     const int32_t* pos, int32_t B, int32_t n_tok,
+                     const mla_cache_t* cache, mla_stream_t stream);
+
+/* Bytes of scratch mla_decode / mla_attend_latent need for this shape on the
+ * current device (depends on the SM count, not on the sequence lengths). */
+size_t mla_workspace_bytes(const mla_dims_t* dims, int32_t B, int32_t q_len);
+
+/* ---------------------------------------------------------------- decode
+ * One absorbed-MLA decode step for B sequences with q_len query tokens each
+ * (q_len = 1 plain decode; 2..4 speculative verify, causal among the new
+ * tokens).  seqlens[b] counts cached tokens INCLUDING the q_len new ones,
+ * which must already be appended; query i sits at position
+ * m = seqlens[b] - q_len + i and attends to keys 0..m.
+ *   q_nope [B][q_len][H][d_n]   content query
+ *   q_rope [B][q_len][H][d_r]   UN-rotated RoPE query (rotated here at m)
+ *   W_UK   [H][d_n][d_c]        k_C = W_UK[h] c      (U in R^{d_h x d_c})
+ *   W_UV   [H][d_v][d_c]        v   = W_UV[h] c
+ *   out    [B][q_len][H][d_v]   written
+ *   workspace: device scratch of at least mla_workspace_bytes(); the call
+ *   owns it until the stream reaches the end of the call.
+ * Steps: absorb (a2), attend in latent space (a3+a4), project (a5). */
+int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_rope,
+               const void* W_UK, const void* W_UV, const mla_cache_t* cache,
+               const int32_t* seqlens, int32_t B, int32_t q_len, void* out,
+               void* workspace, size_t workspace_bytes, mla_stream_t stream);
+
+/* Execution options for tests and tuning.  path: 0 = auto (sm_100a tensor-core
+ * kernels for bf16 V3 geometry, generic CUDA kernels otherwise), 1 = force the
+ * tensor-core path (MLA_ERR_UNSUPPORTED if it cannot run), 2 = force the
+ * generic CUDA path.  num_pairs: CTA pairs of the attention grid (0 = one per
+ * two SMs).  overhead_tiles: scheduling cost charged per sequence, in 64-key
+ * tiles (negative = default). */
+typedef struct {
+    int32_t path;
+    int32_t num_pairs;
+    int32_t overhead_tiles;
+} mla_decode_opts_t;
+
+int mla_decode_ex(const mla_dims_t* dims, const void* q_nope, const void* q_rope,
+                  const void* W_UK, const void* W_UV, const mla_cache_t* cache,
+                  const int32_t* seqlens, int32_t B, int32_t q_len, void* out,
+                  void* workspace, size_t workspace_bytes,
+                  const mla_decode_opts_t* opts, mla_stream_t stream);
+
+/* ---------------------------------------------------------------- steps
+ * The three stages of mla_decode, callable one by one (same layouts).
+ *
+ * a2: q_hat[b][i][h] = [ W_UK[h]^T q_nope[b][i][h]  ||  RoPE(q_rope[b][i][h], m) ]
+ *     q_hat [B][q_len][H][d_c + d_r], dtype of the call. */
+int mla_absorb_query(const mla_dims_t* dims, const void* q_nope, const void* q_rope,
+                     const void* W_UK, const int32_t* seqlens, int32_t B, int32_t q_len,
+                     void* q_hat, const mla_decode_opts_t* opts, mla_stream_t stream);
+
+/* a3+a4: scores s_j = softmax_scale * (q_hat . cache_row_j) over keys
+ * 0..m, softmax, o_lat = sum_j p_j c_KV,j.  o_lat [B][q_len][H][d_c]. */
+int mla_attend_latent(const mla_dims_t* dims, const void* q_hat, const mla_cache_t* cache,
+                      const int32_t* seqlens, int32_t B, int32_t q_len, void* o_lat,
+                      void* workspace, size_t workspace_bytes,
+                      const mla_decode_opts_t* opts, mla_stream_t stream);
+
+/* a5: out[r][h] = W_UV[h] o_lat[r][h] for the `rows` = B*q_len query tokens. */
+int mla_project_out(const mla_dims_t* dims, const void* o_lat, const void* W_UV,
+                    int32_t rows, void* out, const mla_decode_opts_t* opts,
+                    mla_stream_t stream);
+
+/* ---------------------------------------------------------------- status */
+
+/* Synchronises `stream`, returns the device status word in *status (bits
+ * MLA_STATUS_*) and clears it.  Returns MLA_OK, MLA_ERR_CUDA, or
+ * MLA_ERR_DEVICE when the word was non-zero. */
+int mla_device_status(mla_stream_t stream, int32_t* status);
+
+/* Description of the last error on this host thread ("" if none). */
+const char* mla_last_error(void);
+
+/* Name of the path the last mla_decode* / step call on this thread used:
+ * "sm100" or "generic". */
+const char* mla_last_path(void);
+
+/* ABI version (major*100 + minor). */
+int mla_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_H_ */

@@ -1,0 +1,73 @@
+// Internal declarations shared by the translation units of libmla.so.
+// Nothing here is part of the C ABI (that is include/mla.h).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "mla.h"
+
+namespace mla {
+
+// Problem description after host-side validation.
+struct Problem {
+    int H, d_c, d_r, d_n, d_v;
+    int dtype;  // MLA_DTYPE_*
+    float rope_base;
+    float scale;  // softmax scale (already resolved)
+    int B, q_len;
+};
+
+struct CacheView {
+    void* data;
+    int T_max;
+    int64_t stride_b, stride_t;  // elements
+};
+
+// 16-byte-aligned carving of the caller's workspace.
+struct Carve {
+    char* base;
+    size_t off;
+    explicit Carve(void* p) : base(static_cast<char*>(p)), off(0) {}
+    void* take(size_t bytes) {
+        void* r = base ? base + off : nullptr;
+        off += (bytes + 255) & ~size_t(255);
+        return r;
+    }
+};
+
+// Device status word of the current device (set up once per device).
+int* device_status_ptr();
+
+// Number of SMs of the current device.
+int device_sm_count();
+
+// ----------------------------------------------------------- generic CUDA path
+// Plain CUDA-core kernels, any head geometry, fp32 or bf16 storage.
+cudaError_t generic_append(const Problem& p, const void* c_kv, const void* k_rope, const int32_t* pos,
+                           int n_tok, const CacheView& cache, int* status, cudaStream_t st);
+cudaError_t generic_absorb(const Problem& p, const void* q_nope, const void* q_rope, const void* W_UK,
+                           const int32_t* seqlens, void* q_hat, cudaStream_t st);
+cudaError_t generic_attend(const Problem& p, const void* q_hat, const CacheView& cache,
+                           const int32_t* seqlens, void* o_lat, int* status, cudaStream_t st);
+cudaError_t generic_project(const Problem& p, const void* o_lat, const void* W_UV, int rows, void* out,
+                            cudaStream_t st);
+size_t generic_workspace_bytes(const Problem& p);
+
+// ----------------------------------------------------------- sm_100a path
+// bf16 storage, V3 head geometry (d_c 512, d_r 64, d_n 128, d_v 128), H = 128.
+bool sm100_supported(const Problem& p, int q_len);
+cudaError_t sm100_append(const Problem& p, const void* c_kv, const void* k_rope, const int32_t* pos,
+                         int n_tok, const CacheView& cache, int* status, cudaStream_t st);
+cudaError_t sm100_absorb(const Problem& p, const void* q_nope, const void* q_rope, const void* W_UK,
+                         const int32_t* seqlens, void* q_hat, cudaStream_t st);
+cudaError_t sm100_attend(const Problem& p, const void* q_hat, const CacheView& cache, const int32_t* seqlens,
+                         void* o_lat, void* workspace, size_t ws_bytes, int num_pairs, int overhead_tiles,
+                         int* status, cudaStream_t st);
+cudaError_t sm100_project(const Problem& p, const void* o_lat, const void* W_UV, int rows, void* out,
+                          cudaStream_t st);
+size_t sm100_attend_workspace_bytes(const Problem& p, int num_pairs);
+int sm100_default_pairs();
+
+}  // namespace mla
