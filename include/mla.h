@@ -123,17 +123,37 @@ int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_rope,
                const int32_t* seqlens, int32_t B, int32_t q_len, void* out,
                void* workspace, size_t workspace_bytes, mla_stream_t stream);
 
-/* Execution options for tests and tuning.  path: 0 = auto (sm_100a tensor-core
- * kernels for bf16 V3 geometry, generic CUDA kernels otherwise), 1 = force the
- * tensor-core path (MLA_ERR_UNSUPPORTED if it cannot run), 2 = force the
- * generic CUDA path.  num_pairs: CTA pairs of the attention grid (0 = one per
- * two SMs).  overhead_tiles: scheduling cost charged per sequence, in 64-key
- * tiles (negative = default). */
+/* Execution options for tests, tuning and profiling.
+ *   path: 0 = auto (sm_100a tensor-core kernels for bf16 V3 geometry, generic
+ *         CUDA kernels otherwise), 1 = force the tensor-core path
+ *         (MLA_ERR_UNSUPPORTED if it cannot run), 2 = force the generic path.
+ *   num_pairs: CTA pairs (clusters) of the attention grid (0 = one per two SMs).
+ *   overhead_tiles: scheduling cost charged per sequence, in 64-key tiles
+ *         (negative = default).
+ *   events / n_events: optional caller-created cudaEvent_t handles; when
+ *         n_events >= MLA_NUM_EVENTS, mla_decode_ex records them on `stream`
+ *         at the stage boundaries listed below, so a caller can time each
+ *         kernel with cudaEventElapsedTime.  The library does not own them.
+ *   All-zero options (path 0, num_pairs 0, overhead_tiles 0, no events) are valid. */
 typedef struct {
     int32_t path;
     int32_t num_pairs;
     int32_t overhead_tiles;
+    int32_t n_events;
+    void* const* events;
 } mla_decode_opts_t;
+
+/* Event slots recorded by mla_decode_ex (sm_100a path; the generic path
+ * records 0, 1 before/after absorb and 5 at the end, with 2..4 after attend). */
+enum {
+    MLA_EV_START = 0,        /* before the absorb GEMM */
+    MLA_EV_ABSORB_DONE = 1,  /* after absorb (before the split planner) */
+    MLA_EV_ATTEND_BEGIN = 2, /* before the attention kernel */
+    MLA_EV_ATTEND_END = 3,   /* after the attention kernel (before the split combine) */
+    MLA_EV_COMBINE_DONE = 4, /* after the split combine (before W_UV) */
+    MLA_EV_END = 5,          /* after the W_UV projection */
+    MLA_NUM_EVENTS = 6
+};
 
 int mla_decode_ex(const mla_dims_t* dims, const void* q_nope, const void* q_rope,
                   const void* W_UK, const void* W_UV, const mla_cache_t* cache,

@@ -21,6 +21,8 @@ LIB_PATH = os.path.join(_HERE, "libmla.so")
 MLA_DTYPE_BF16, MLA_DTYPE_F32 = 0, 1
 PATH_AUTO, PATH_SM100, PATH_GENERIC = 0, 1, 2
 STATUS_BAD_POS, STATUS_BAD_SEQLEN, STATUS_TIMEOUT = 1, 2, 4
+NUM_EVENTS = 6
+EV_START, EV_ABSORB_DONE, EV_ATTEND_BEGIN, EV_ATTEND_END, EV_COMBINE_DONE, EV_END = range(6)
 ERRORS = {-1: "MLA_ERR_ARG", -2: "MLA_ERR_SHAPE", -3: "MLA_ERR_ALIGN", -4: "MLA_ERR_CUDA",
           -5: "MLA_ERR_TIMEOUT", -6: "MLA_ERR_DEVICE", -7: "MLA_ERR_WORKSPACE", -8: "MLA_ERR_UNSUPPORTED"}
 
@@ -42,7 +44,8 @@ class Cache(ctypes.Structure):
 
 
 class Opts(ctypes.Structure):
-    _fields_ = [("path", ctypes.c_int32), ("num_pairs", ctypes.c_int32), ("overhead_tiles", ctypes.c_int32)]
+    _fields_ = [("path", ctypes.c_int32), ("num_pairs", ctypes.c_int32), ("overhead_tiles", ctypes.c_int32),
+                ("n_events", ctypes.c_int32), ("events", ctypes.POINTER(ctypes.c_void_p))]
 
 
 class MLAError(RuntimeError):
@@ -128,8 +131,15 @@ class Library:
         return Cache(cache.data_ptr(), cache.shape[0], cache.shape[1], cache.stride(0), cache.stride(1))
 
     @staticmethod
-    def opts(path=PATH_AUTO, num_pairs=0, overhead_tiles=-1) -> Opts:
-        return Opts(path, num_pairs, overhead_tiles)
+    def opts(path=PATH_AUTO, num_pairs=0, overhead_tiles=-1, events=None) -> Opts:
+        """``events``: MLA_NUM_EVENTS recorded torch.cuda.Event objects (stage timing)."""
+        o = Opts(path, num_pairs, overhead_tiles, 0, None)
+        if events is not None:
+            arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
+            o.events = ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p))
+            o.n_events = len(events)
+            o._keep = arr  # keep the array alive as long as the options
+        return o
 
     def last_path(self) -> str:
         return self.lib.mla_last_path().decode()

@@ -310,18 +310,31 @@ int mla_decode_ex(const mla_dims_t* dims, const void* q_nope, const void* q_rope
     void* q_hat = ws + L.q_hat;
     void* o_lat = ws + L.o_lat;
     const cudaStream_t st = (cudaStream_t)stream;
+    Events ev;
+    if (opts && opts->events && opts->n_events >= MLA_NUM_EVENTS) {
+        for (int i = 0; i < MLA_NUM_EVENTS; ++i) ev.ev[i] = (cudaEvent_t)opts->events[i];
+        ev.on = true;
+    }
     cudaError_t e;
+    ev.record(MLA_EV_START, st);
     if (fast) {
         e = sm100_absorb(p, q_nope, q_rope, W_UK, seqlens, q_hat, st);
+        ev.record(MLA_EV_ABSORB_DONE, st);
         if (e == cudaSuccess)
             e = sm100_attend(p, q_hat, cv, seqlens, o_lat, ws + L.attend, L.total - L.attend, pairs,
-                             opts ? opts->overhead_tiles : -1, status, st);
+                             opts ? opts->overhead_tiles : -1, status, st, &ev);
+        ev.record(MLA_EV_COMBINE_DONE, st);
         if (e == cudaSuccess) e = sm100_project(p, o_lat, W_UV, B * q_len, out, st);
     } else {
         e = generic_absorb(p, q_nope, q_rope, W_UK, seqlens, q_hat, st);
+        ev.record(MLA_EV_ABSORB_DONE, st);
         if (e == cudaSuccess) e = generic_attend(p, q_hat, cv, seqlens, o_lat, status, st);
+        ev.record(MLA_EV_ATTEND_BEGIN, st);
+        ev.record(MLA_EV_ATTEND_END, st);
+        ev.record(MLA_EV_COMBINE_DONE, st);
         if (e == cudaSuccess) e = generic_project(p, o_lat, W_UV, B * q_len, out, st);
     }
+    ev.record(MLA_EV_END, st);
     t_path = fast ? "sm100" : "generic";
     return e == cudaSuccess ? MLA_OK : cuda_fail(e, "decode launch");
 }

@@ -19,6 +19,15 @@ struct Problem {
     int B, q_len;
 };
 
+// Optional stage-boundary events of one decode call (see MLA_EV_* in mla.h).
+struct Events {
+    cudaEvent_t ev[MLA_NUM_EVENTS];
+    bool on = false;
+    void record(int i, cudaStream_t st) const {
+        if (on) cudaEventRecord(ev[i], st);
+    }
+};
+
 struct CacheView {
     void* data;
     int T_max;
@@ -64,7 +73,7 @@ cudaError_t sm100_absorb(const Problem& p, const void* q_nope, const void* q_rop
                          const int32_t* seqlens, void* q_hat, cudaStream_t st);
 cudaError_t sm100_attend(const Problem& p, const void* q_hat, const CacheView& cache, const int32_t* seqlens,
                          void* o_lat, void* workspace, size_t ws_bytes, int num_pairs, int overhead_tiles,
-                         int* status, cudaStream_t st);
+                         int* status, cudaStream_t st, const Events* events = nullptr);
 cudaError_t sm100_project(const Problem& p, const void* o_lat, const void* W_UV, int rows, void* out,
                           cudaStream_t st);
 size_t sm100_attend_workspace_bytes(const Problem& p, int num_pairs);

@@ -77,10 +77,21 @@ __global__ void append_v3_kernel(const __nv_bfloat16* __restrict__ c_kv, const _
     reinterpret_cast<__nv_bfloat162*>(row + kLat)[lane] = __floats2bfloat162_rn(y0, y1);
 }
 
+// Opt a kernel into more than 48 KB of dynamic shared memory, once per device
+// and call site (`done` is that site's own flag array), so that later calls,
+// including ones under stream capture, make no attribute calls.
+constexpr int kMaxDev = 64;
 template <typename K>
-cudaError_t set_smem(K kernel, int bytes) {
-    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+cudaError_t set_smem(K kernel, int bytes, bool (&done)[kMaxDev]) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < kMaxDev && done[dev]) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && dev >= 0 && dev < kMaxDev) done[dev] = true;
+    return e;
 }
+bool g_smem_absorb[kMaxDev], g_smem_project[kMaxDev], g_smem_attend[kMaxDev];
 
 constexpr int kAbsorbStages = 2;
 constexpr int kProjStages = 4;
@@ -126,7 +137,7 @@ cudaError_t sm100_absorb(const Problem& p, const void* q_nope, const void* q_rop
         return cudaErrorInvalidValue;
     using Cfg = GemmCfg<2, 256, true, kAbsorbStages, true>;
     auto kern = head_gemm_kernel<2, 256, true, kAbsorbStages, true>;
-    cudaError_t e = set_smem(kern, Cfg::kSmem);
+    cudaError_t e = set_smem(kern, Cfg::kSmem, g_smem_absorb);
     if (e != cudaSuccess) return e;
     GemmArgs a;
     a.rows = rows;
@@ -157,7 +168,7 @@ cudaError_t sm100_project(const Problem& p, const void* o_lat, const void* W_UV,
         return cudaErrorInvalidValue;
     using Cfg = GemmCfg<8, kProjNT, false, kProjStages, false>;
     auto kern = head_gemm_kernel<8, kProjNT, false, kProjStages, false>;
-    cudaError_t e = set_smem(kern, Cfg::kSmem);
+    cudaError_t e = set_smem(kern, Cfg::kSmem, g_smem_project);
     if (e != cudaSuccess) return e;
     GemmArgs a;
     memset(&a, 0, sizeof(a));
@@ -192,7 +203,7 @@ size_t sm100_attend_workspace_bytes(const Problem& p, int num_pairs) {
 
 cudaError_t sm100_attend(const Problem& p, const void* q_hat, const CacheView& cache, const int32_t* seqlens,
                          void* o_lat, void* workspace, size_t ws_bytes, int num_pairs, int overhead_tiles,
-                         int* status, cudaStream_t st) {
+                         int* status, cudaStream_t st, const Events* events) {
     const int clusters = num_pairs;
     size_t off_part, off_lse;
     const size_t need = attend_layout(p, clusters, &off_part, &off_lse);
@@ -216,7 +227,7 @@ cudaError_t sm100_attend(const Problem& p, const void* q_hat, const CacheView& c
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
 
-    e = set_smem(mla_attend_kernel, kAttSmem);
+    e = set_smem(mla_attend_kernel, kAttSmem, g_smem_attend);
     if (e != cudaSuccess) return e;
     AttendArgs a;
     a.plan = plan;
@@ -243,8 +254,10 @@ cudaError_t sm100_attend(const Problem& p, const void* q_hat, const CacheView& c
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    if (events) events->record(MLA_EV_ATTEND_BEGIN, st);
     e = cudaLaunchKernelEx(&cfg, mla_attend_kernel, mCL, mCR, mQL, mQR, a);
     if (e != cudaSuccess) return e;
+    if (events) events->record(MLA_EV_ATTEND_END, st);
 
     const int warps = p.B * p.q_len * kHeads;
     mla_combine_kernel<<<(warps * 32 + 255) / 256, 256, 0, st>>>(plan, a.part_o, a.part_lse, p.q_len,
