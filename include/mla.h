@@ -161,6 +161,34 @@ int mla_decode_ex(const mla_dims_t* dims, const void* q_nope, const void* q_rope
                   void* workspace, size_t workspace_bytes,
                   const mla_decode_opts_t* opts, mla_stream_t stream);
 
+/* ---------------------------------------------------------------- no-allocation decode
+ * The same decode step as mla_decode for callers that cannot allocate device
+ * memory: code whose device memory is owned by another allocator (a server or
+ * framework that does not let plug-ins call cudaMalloc), or a serving loop
+ * that must not allocate after start-up because cudaMalloc / cudaFree can
+ * synchronise the device.  The paper has no counterpart; this is an
+ * interface convenience of this library.
+ *
+ * Arguments, layouts and results are those of mla_decode, without the
+ * workspace: the scratch is a fixed 64 MiB array inside the library's device
+ * image, which every GPU that loads the library keeps until the process
+ * exits.  A batch whose mla_workspace_bytes() exceeds 64 MiB is rejected with
+ * MLA_ERR_WORKSPACE before anything is launched; on a 148-SM B200 the limit
+ * is 88 sequences at q_len = 1, 26 at q_len = 2, 5 at q_len = 3 (q_len = 4
+ * does not fit).  The call allocates nothing
+ * and calls no allocating routine.
+ *
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current); make that first call
+ * before any stream capture.  All calls on a device share the one array and
+ * it keeps the last call's contents (nothing needs to start at zero); calls
+ * that overlap on the GPU, on different streams or threads, race on it and
+ * must be ordered by the caller. */
+int mla_decode_no_alloc(const mla_dims_t* dims, const void* q_nope, const void* q_rope,
+                        const void* W_UK, const void* W_UV, const mla_cache_t* cache,
+                        const int32_t* seqlens, int32_t B, int32_t q_len, void* out,
+                        mla_stream_t stream);
+
 /* ---------------------------------------------------------------- steps
  * The three stages of mla_decode, callable one by one (same layouts).
  *

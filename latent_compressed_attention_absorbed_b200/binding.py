@@ -29,7 +29,7 @@ ERRORS = {-1: "MLA_ERR_ARG", -2: "MLA_ERR_SHAPE", -3: "MLA_ERR_ALIGN", -4: "MLA_
 # Every symbol the header declares (checked by the CPU test suite).
 EXPORTS = ["mla_append_cache", "mla_workspace_bytes", "mla_decode", "mla_decode_ex", "mla_absorb_query",
            "mla_attend_latent", "mla_project_out", "mla_device_status", "mla_last_error", "mla_last_path",
-           "mla_version"]
+           "mla_version", "mla_decode_no_alloc"]
 
 
 class Dims(ctypes.Structure):
@@ -63,6 +63,8 @@ _SIGS = {
                     ctypes.c_size_t, _P], ctypes.c_int),
     "mla_decode_ex": ([ctypes.POINTER(Dims), _P, _P, _P, _P, ctypes.POINTER(Cache), _P, _I, _I, _P, _P,
                        ctypes.c_size_t, ctypes.POINTER(Opts), _P], ctypes.c_int),
+    "mla_decode_no_alloc": ([ctypes.POINTER(Dims), _P, _P, _P, _P, ctypes.POINTER(Cache), _P, _I, _I, _P, _P],
+                            ctypes.c_int),
     "mla_absorb_query": ([ctypes.POINTER(Dims), _P, _P, _P, _P, _I, _I, _P, ctypes.POINTER(Opts), _P], ctypes.c_int),
     "mla_attend_latent": ([ctypes.POINTER(Dims), _P, ctypes.POINTER(Cache), _P, _I, _I, _P, _P, ctypes.c_size_t,
                            ctypes.POINTER(Opts), _P], ctypes.c_int),
@@ -179,6 +181,20 @@ class Library:
         self._check(self.lib.mla_decode_ex(ctypes.byref(dims), _ptr(q_nope), _ptr(q_rope), _ptr(W_UK), _ptr(W_UV),
                                            ctypes.byref(cd), _ptr(seqlens), B, q_len, _ptr(out), _ptr(workspace),
                                            workspace.numel(), ctypes.byref(o), _stream(stream)))
+        return out
+
+    def decode_no_alloc(self, dims: Dims, q_nope, q_rope, W_UK, W_UV, cache, seqlens, out=None, stream=None):
+        """Same step as decode() using the library's static device scratch (no workspace argument)."""
+        for t, n in ((q_nope, "q_nope"), (q_rope, "q_rope"), (W_UK, "W_UK"), (W_UV, "W_UV")):
+            _need(t, n)
+        _need(seqlens, "seqlens", dtype=torch.int32, ndim=1)
+        B, q_len = q_nope.shape[0], q_nope.shape[1]
+        if out is None:
+            out = torch.empty((B, q_len, dims.H, dims.d_v), dtype=q_nope.dtype, device=q_nope.device)
+        cd = self.cache_desc(cache)
+        self._check(self.lib.mla_decode_no_alloc(ctypes.byref(dims), _ptr(q_nope), _ptr(q_rope), _ptr(W_UK),
+                                                 _ptr(W_UV), ctypes.byref(cd), _ptr(seqlens), B, q_len, _ptr(out),
+                                                 _stream(stream)))
         return out
 
     def absorb_query(self, dims: Dims, q_nope, q_rope, W_UK, seqlens, out=None, opts=None, stream=None):

@@ -129,6 +129,14 @@ DecodeLayout decode_layout(const Problem& p, bool fast, int pairs) {
 
 }  // namespace
 
+int set_error(int code, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(t_err, sizeof(t_err), fmt, ap);
+    va_end(ap);
+    return code;
+}
+
 int* device_status_ptr() {
     const int d = current_device();
     if (d < 0 || d >= kMaxDevices) return nullptr;

@@ -46,6 +46,9 @@ struct Carve {
     }
 };
 
+// Records the thread's last-error text (read by mla_last_error) and returns `code`.
+int set_error(int code, const char* fmt, ...);
+
 // Device status word of the current device (set up once per device).
 int* device_status_ptr();
 
