@@ -11,6 +11,14 @@
 #include "sm100_attend.cuh"
 #include "sm100_gemm.cuh"
 
+#ifdef MLA_TRACE
+// Copies the attention kernel's timing trace (4096 tiles x 16 stamps) to host
+// memory; only in builds compiled with -DMLA_TRACE.
+extern "C" int mla_trace_read(void* host, size_t bytes) {
+    return cudaMemcpyFromSymbol(host, mla::sm100::g_mla_trace, bytes) == cudaSuccess ? 0 : -4;
+}
+#endif
+
 namespace mla {
 
 using namespace sm100;
@@ -210,16 +218,10 @@ cudaError_t sm100_attend(const Problem& p, const void* q_hat, const CacheView& c
     if (ws_bytes < need) return cudaErrorInvalidValue;
     char* ws = static_cast<char*>(workspace);
     Plan* plan = reinterpret_cast<Plan*>(ws);
-    const int rows = p.B * p.q_len;
-
-    CUtensorMap mCL, mCR, mQL, mQR;
+    CUtensorMap mCL, mCR;
     const uint64_t sb = (uint64_t)cache.stride_b * 2, stt = (uint64_t)cache.stride_t * 2;
     if (!make_map(&mCL, cache.data, kRow, cache.T_max, p.B, stt, sb, 64, kNk, 1, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&mCR, cache.data, kRow, cache.T_max, p.B, stt, sb, 32, kNk, 1, CU_TENSOR_MAP_SWIZZLE_64B) ||
-        !make_map(&mQL, q_hat, kRow, kHeads, rows, kRow * 2, (uint64_t)kHeads * kRow * 2, 64, kHeads, 1,
-                  CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&mQR, q_hat, kRow, kHeads, rows, kRow * 2, (uint64_t)kHeads * kRow * 2, 32, kHeads, 1,
-                  CU_TENSOR_MAP_SWIZZLE_64B))
+        !make_map(&mCR, cache.data, kRow, cache.T_max, p.B, stt, sb, 32, kNk, 1, CU_TENSOR_MAP_SWIZZLE_64B))
         return cudaErrorInvalidValue;
 
     const int ovh = overhead_tiles < 0 ? 2 : overhead_tiles;
@@ -235,6 +237,7 @@ cudaError_t sm100_attend(const Problem& p, const void* q_hat, const CacheView& c
     a.q_len = p.q_len;
     a.T_max = cache.T_max;
     a.scale_log2 = p.scale * 1.4426950408889634f;
+    a.q_hat = (const __nv_bfloat16*)q_hat;
     a.o_lat = (__nv_bfloat16*)o_lat;
     a.part_o = reinterpret_cast<float*>(ws + off_part);
     a.part_lse = reinterpret_cast<float*>(ws + off_lse);
@@ -255,7 +258,7 @@ cudaError_t sm100_attend(const Problem& p, const void* q_hat, const CacheView& c
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     if (events) events->record(MLA_EV_ATTEND_BEGIN, st);
-    e = cudaLaunchKernelEx(&cfg, mla_attend_kernel, mCL, mCR, mQL, mQR, a);
+    e = cudaLaunchKernelEx(&cfg, mla_attend_kernel, mCL, mCR, a);
     if (e != cudaSuccess) return e;
     if (events) events->record(MLA_EV_ATTEND_END, st);
 

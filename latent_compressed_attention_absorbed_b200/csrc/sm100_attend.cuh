@@ -50,21 +50,24 @@ constexpr int kRow = kLat + kRope;
 constexpr int kHalfLat = 256;
 constexpr int kHalfRope = 32;
 
-// Shared-memory map (offsets from a 1024-aligned base).
-constexpr int kQBytes = kHeads * 128 * 4 + kHeads * 64;    // 4 SW128 chunks + 1 SW64 chunk = 73728
+// Shared-memory map (offsets from a 1024-aligned base): a ring of cache
+// tiles (each: 4 SW128 chunks of 64 keys x 64 latent columns, then one SW64
+// chunk of 64 keys x 32 RoPE columns) and two buffers in which this CTA
+// publishes its partial scores for the peer to read.  Q-hat and P live in
+// tensor memory.
 constexpr int kTileBytes = kNk * 128 * 4 + kNk * 64;       // 36864
-constexpr int kStages = 2;
-constexpr int kPBytes = kHeads * 128;                      // 128 x 64 bf16, SW128
-constexpr int kXBytes = kHeads * kNk * 4;                  // 128 x 64 fp32
-constexpr int kOffQ = 0;
-constexpr int kOffTiles = kOffQ + kQBytes;
-constexpr int kOffP = kOffTiles + kStages * kTileBytes;
-constexpr int kOffX = kOffP + kPBytes;
-constexpr int kOffBars = kOffX + kXBytes;
+constexpr int kStages = 5;
+constexpr int kXBytes = kHeads * kNk * 2;                  // 128 x 64 fp16 partial scores
+constexpr int kOffTiles = 0;
+constexpr int kOffX = kOffTiles + kStages * kTileBytes;    // two publish buffers
+constexpr int kOffBars = kOffX + 2 * kXBytes;
 constexpr int kAttSmem = kOffBars + 256 + 1024;
+// Tensor-memory map (columns of 32 bits, 128 lanes = heads).
 constexpr int kTmemCols = 512;
-constexpr int kTmemO = 0;
-constexpr int kTmemS = 256;
+constexpr int kTmemO = 0;      // O: 256 fp32 latent columns of this half
+constexpr int kTmemS = 256;    // S: 64 fp32 scores (partial, this half's 288 columns)
+constexpr int kTmemP = 320;    // P: 64 bf16 probabilities, two per column
+constexpr int kTmemQ = 352;    // Q-hat half: 256 latent + 32 RoPE bf16, two per column (144 columns)
 constexpr int kAttThreads = 192;
 
 // Barrier indices (8 bytes each) inside the barrier block.
@@ -79,10 +82,26 @@ enum {
     kBarPFree,
     kBarOFull,
     kBarOFree,
-    kBarXFull,
-    kBarXEmpty,
+    kBarXReady0,  // peer has published its partial S in its buffer 0 / 1
+    kBarXReady1,
+    kBarXRead0,   // peer has finished reading our buffer 0 / 1
+    kBarXRead1,
     kNumBars
 };
+
+// Optional timing trace (compile with -DMLA_TRACE): clock64 stamps of the
+// first CTA at 16 fixed points of every tile, read back by mla_trace_read.
+#ifdef MLA_TRACE
+__device__ unsigned long long g_mla_trace[4096][16];
+#define MLA_TRACE_POINT(ev, n)                                                 \
+    do {                                                                       \
+        if (cl == 0 && crank == 0 && (n) < 4096) g_mla_trace[(n)][(ev)] = clock64(); \
+    } while (0)
+#else
+#define MLA_TRACE_POINT(ev, n) \
+    do {                       \
+    } while (0)
+#endif
 
 // Scheduling plan written by the plan kernel into the workspace.
 struct Plan {
@@ -140,27 +159,43 @@ struct SegIter {
     }
 };
 
+// Flat walk over the tiles of a cluster's pieces, with the piece's bounds.
+struct TileWalk {
+    SegIter it;
+    int seq, k0, k1, t, seg;
+    bool whole, valid;
+    __device__ void init(const Plan* plan, int cl) {
+        it.init(plan, cl);
+        seg = 0;
+        valid = it.next(seq, k0, k1, whole);
+        t = k0;
+    }
+    __device__ bool first() const { return t == k0; }
+    __device__ bool last() const { return t == k1 - 1; }
+    __device__ void advance() {
+        if (++t >= k1) {
+            valid = it.next(seq, k0, k1, whole);
+            t = k0;
+            ++seg;
+        }
+    }
+};
+
 struct AttendArgs {
     const Plan* plan;
     const int32_t* seqlens;
     int q_len;
     int T_max;
     float scale_log2;             // softmax_scale * log2(e)
+    const __nv_bfloat16* q_hat;   // [B][q_len][128][576]
     __nv_bfloat16* o_lat;         // [B][q_len][128][512]
     float* part_o;                // [slots][q_len][128][512]
     float* part_lse;              // [slots][q_len][128]
     int* status;
 };
 
-// Row r of a SW128 K-major tile (128-byte rows, 8-row atoms): byte offset of
-// 16-byte chunk k.
-__device__ __forceinline__ uint32_t sw128_off(int r, int k) {
-    return (uint32_t)(r * 128 + ((k ^ (r & 7)) << 4));
-}
-
 __global__ void __launch_bounds__(kAttThreads, 1)
     mla_attend_kernel(const __grid_constant__ CUtensorMap mapCacheLat, const __grid_constant__ CUtensorMap mapCacheRope,
-                      const __grid_constant__ CUtensorMap mapQLat, const __grid_constant__ CUtensorMap mapQRope,
                       AttendArgs args) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -183,7 +218,7 @@ __global__ void __launch_bounds__(kAttThreads, 1)
             mbar_init(bar(kBarFull0 + s), 1);
             mbar_init(bar(kBarEmpty0 + s), 1);
         }
-        mbar_init(bar(kBarQFull), 1);
+        mbar_init(bar(kBarQFull), 4);
         mbar_init(bar(kBarQEmpty), 1);
         mbar_init(bar(kBarSFull), 1);
         mbar_init(bar(kBarSFree), 4);
@@ -191,14 +226,14 @@ __global__ void __launch_bounds__(kAttThreads, 1)
         mbar_init(bar(kBarPFree), 1);
         mbar_init(bar(kBarOFull), 1);
         mbar_init(bar(kBarOFree), 4);
-        mbar_init(bar(kBarXFull), 1);
-        mbar_init(bar(kBarXEmpty), 4);
+        mbar_init(bar(kBarXReady0), 4);
+        mbar_init(bar(kBarXReady1), 4);
+        mbar_init(bar(kBarXRead0), 4);
+        mbar_init(bar(kBarXRead1), 4);
         *abort_flag = 0;
         fence_mbar_init();
         prefetch_tensormap(&mapCacheLat);
         prefetch_tensormap(&mapCacheRope);
-        prefetch_tensormap(&mapQLat);
-        prefetch_tensormap(&mapQRope);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, kTmemCols);
@@ -210,281 +245,332 @@ __global__ void __launch_bounds__(kAttThreads, 1)
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(base_ptr + kOffBars + 8 * kNumBars);
 
-    SegIter it;
-    it.init(args.plan, cl);
-    int seq, k0, k1;
-    bool whole;
-
     if (warp == 0) {
-        // ======================================================== TMA producer
+        // ======================================================== TMA producer (runs up to kStages tiles ahead)
         if (lane == 0) {
-            int n = 0, s_cnt = 0;
-            while (!*abort_flag && it.next(seq, k0, k1, whole)) {
-                if (s_cnt > 0 && !mbar_wait(bar(kBarQEmpty), (s_cnt - 1) & 1)) { *abort_flag = 1; break; }
-                const int u = seq * q_len + qi;
-                mbar_arrive_expect_tx(bar(kBarQFull), kQBytes);
-                for (int c = 0; c < 4; ++c)
-                    tma_load_3d(base + kOffQ + c * (kHeads * 128), &mapQLat, bar(kBarQFull),
-                                half * kHalfLat + 64 * c, 0, u);
-                tma_load_3d(base + kOffQ + 4 * (kHeads * 128), &mapQRope, bar(kBarQFull),
-                            kLat + half * kHalfRope, 0, u);
-                for (int t = k0; t < k1; ++t, ++n) {
-                    const int st = n % kStages;
-                    if (n >= kStages && !mbar_wait(bar(kBarEmpty0 + st), ((n / kStages) - 1) & 1)) {
-                        *abort_flag = 1;
-                        break;
-                    }
-                    const uint32_t dst = base + kOffTiles + st * kTileBytes;
-                    mbar_arrive_expect_tx(bar(kBarFull0 + st), kTileBytes);
-                    for (int c = 0; c < 4; ++c)
-                        tma_load_3d(dst + c * (kNk * 128), &mapCacheLat, bar(kBarFull0 + st),
-                                    half * kHalfLat + 64 * c, t * kNk, seq);
-                    tma_load_3d(dst + 4 * (kNk * 128), &mapCacheRope, bar(kBarFull0 + st),
-                                kLat + half * kHalfRope, t * kNk, seq);
+            TileWalk w;
+            w.init(args.plan, cl);
+            for (int n = 0; w.valid && !*abort_flag; ++n, w.advance()) {
+                const int st = n % kStages;
+                if (n >= kStages && !mbar_wait(bar(kBarEmpty0 + st), ((n / kStages) - 1) & 1)) {
+                    *abort_flag = 1;
+                    break;
                 }
-                ++s_cnt;
+                const uint32_t dst = base + kOffTiles + st * kTileBytes;
+                mbar_arrive_expect_tx(bar(kBarFull0 + st), kTileBytes);
+                for (int c = 0; c < 4; ++c)
+                    tma_load_3d(dst + c * (kNk * 128), &mapCacheLat, bar(kBarFull0 + st), half * kHalfLat + 64 * c,
+                                w.t * kNk, w.seq);
+                tma_load_3d(dst + 4 * (kNk * 128), &mapCacheRope, bar(kBarFull0 + st), kLat + half * kHalfRope,
+                            w.t * kNk, w.seq);
+                MLA_TRACE_POINT(0, n);
             }
         }
     } else if (warp == 1) {
         // ======================================================== MMA issuer (whole warp waits, lane 0 issues)
         constexpr uint32_t idS = idesc_bf16_f32(128, kNk, false, false);
         constexpr uint32_t idO = idesc_bf16_f32(128, kHalfLat, false, true);
-        int n = 0, s_cnt = 0;
         bool ok = true;
-        while (ok && !*abort_flag && it.next(seq, k0, k1, whole)) {
-            const int T_b = args.seqlens[seq];
-            if (!mbar_wait(bar(kBarQFull), s_cnt & 1)) { ok = false; break; }
-            const int n_first = n;
-            for (int t = k0; t < k1 && ok; ++t, ++n) {
-                const int st = n % kStages;
-                const uint32_t tile = base + kOffTiles + st * kTileBytes;
-                if (!mbar_wait(bar(kBarFull0 + st), (n / kStages) & 1)) { ok = false; break; }
-                const int valid = T_b - t * kNk;
-                if (valid < kNk) {
-                    // Rows at or beyond T_b hold no cached token: zero them so
-                    // that masked (p = 0) rows cannot inject NaN/Inf into P.C.
-                    const int r0 = valid < 0 ? 0 : valid;
-                    for (int r = r0 + (lane >> 3); r < kNk; r += 4) {
-                        for (int c = 0; c < 4; ++c)
-                            st_shared_v4(tile + c * (kNk * 128) + r * 128 + (lane & 7) * 16, 0, 0, 0, 0);
-                        if ((lane & 7) < 4) st_shared_v4(tile + 4 * (kNk * 128) + r * 64 + (lane & 7) * 16, 0, 0, 0, 0);
-                    }
-                    fence_proxy_async_smem();
-                }
-                __syncwarp();
-                // S(n) needs the softmax warps to have read S(n-1) out of TMEM.
-                if (n > 0 && !mbar_wait(bar(kBarSFree), (n - 1) & 1)) { ok = false; break; }
-                tc_fence_after();
-                if (lane == 0) {
-                    // S = Qhat_half . C_half^T : 4 latent chunks x 4 K-steps + 2 RoPE K-steps
-                    for (int c = 0; c < 4; ++c)
-                        for (int k = 0; k < 4; ++k) {
-                            const uint64_t ad = smem_desc(base + kOffQ + c * (kHeads * 128) + 32 * k, 16, 1024, kSw128);
-                            const uint64_t bd = smem_desc(tile + c * (kNk * 128) + 32 * k, 16, 1024, kSw128);
-                            mma_f16_ss(tmem + kTmemS, ad, bd, idS, (c | k) ? 1u : 0u);
-                        }
-                    for (int k = 0; k < 2; ++k) {
-                        const uint64_t ad = smem_desc(base + kOffQ + 4 * (kHeads * 128) + 32 * k, 16, 512, kSw64);
-                        const uint64_t bd = smem_desc(tile + 4 * (kNk * 128) + 32 * k, 16, 512, kSw64);
-                        mma_f16_ss(tmem + kTmemS, ad, bd, idS, 1u);
-                    }
-                    mma_commit(bar(kBarSFull));
-                }
-                __syncwarp();
-                if (n > n_first) {
-                    // O += P(n-1) . C(n-1)
-                    const int pn = n - 1;
-                    if (!mbar_wait(bar(kBarPFull), pn & 1)) { ok = false; break; }
-                    if (pn == n_first && s_cnt > 0 && !mbar_wait(bar(kBarOFree), (s_cnt - 1) & 1)) { ok = false; break; }
-                    tc_fence_after();
-                    if (lane == 0) {
-                        const uint32_t ptile = base + kOffTiles + (pn % kStages) * kTileBytes;
-                        for (int k = 0; k < 4; ++k) {
-                            const uint64_t ad = smem_desc(base + kOffP + 32 * k, 16, 1024, kSw128);
-                            const uint64_t bd = smem_desc(ptile + 2048 * k, kNk * 128, 1024, kSw128);
-                            mma_f16_ss(tmem + kTmemO, ad, bd, idO, (pn > n_first || k > 0) ? 1u : 0u);
-                        }
-                        mma_commit(bar(kBarPFree));
-                        mma_commit(bar(kBarEmpty0 + (pn % kStages)));
-                    }
-                    __syncwarp();
-                }
+        // O(g) += P(g) . C(g); its first K-step overwrites O at the start of a piece.
+        auto issue_O = [&](int g, bool first_in_seg, bool last_in_seg) {
+            const uint32_t ptile = base + kOffTiles + (g % kStages) * kTileBytes;
+            for (int k = 0; k < 4; ++k) {
+                const uint64_t bd = smem_desc(ptile + 2048 * k, kNk * 128, 1024, kSw128);
+                mma_f16_ts(tmem + kTmemO, tmem + kTmemP + 8 * k, bd, idO, (!first_in_seg || k > 0) ? 1u : 0u);
             }
-            if (!ok) break;
-            // All S MMAs of this segment are issued: Q-hat may be reloaded once they finish.
-            if (lane == 0) mma_commit(bar(kBarQEmpty));
-            const int pn = n - 1;
-            if (!mbar_wait(bar(kBarPFull), pn & 1)) { ok = false; break; }
-            if (pn == n_first && s_cnt > 0 && !mbar_wait(bar(kBarOFree), (s_cnt - 1) & 1)) { ok = false; break; }
-            tc_fence_after();
-            if (lane == 0) {
-                const uint32_t ptile = base + kOffTiles + (pn % kStages) * kTileBytes;
-                for (int k = 0; k < 4; ++k) {
-                    const uint64_t ad = smem_desc(base + kOffP + 32 * k, 16, 1024, kSw128);
-                    const uint64_t bd = smem_desc(ptile + 2048 * k, kNk * 128, 1024, kSw128);
-                    mma_f16_ss(tmem + kTmemO, ad, bd, idO, (pn > n_first || k > 0) ? 1u : 0u);
+            mma_commit(bar(kBarPFree));
+            mma_commit(bar(kBarEmpty0 + (g % kStages)));
+            if (last_in_seg) mma_commit(bar(kBarOFull));
+        };
+        TileWalk w;
+        w.init(args.plan, cl);
+        bool prev_first = false, prev_last = false;
+        int prev_seg = 0;
+        int g = 0;
+        for (; w.valid && ok && !*abort_flag; ++g, w.advance()) {
+            const int T_b = args.seqlens[w.seq];
+            if (w.first() && !mbar_wait(bar(kBarQFull), w.seg & 1)) { ok = false; break; }
+            const int st = g % kStages;
+            const uint32_t tile = base + kOffTiles + st * kTileBytes;
+            if (!mbar_wait(bar(kBarFull0 + st), (g / kStages) & 1)) { ok = false; break; }
+            MLA_TRACE_POINT(1, g);
+            const int valid = T_b - w.t * kNk;
+            if (valid < kNk) {
+                // Rows at or beyond T_b hold no cached token: zero them so that
+                // masked (p = 0) rows cannot inject NaN/Inf into P.C.
+                const int r0 = valid < 0 ? 0 : valid;
+                for (int r = r0 + (lane >> 3); r < kNk; r += 4) {
+                    for (int c = 0; c < 4; ++c)
+                        st_shared_v4(tile + c * (kNk * 128) + r * 128 + (lane & 7) * 16, 0, 0, 0, 0);
+                    if ((lane & 7) < 4) st_shared_v4(tile + 4 * (kNk * 128) + r * 64 + (lane & 7) * 16, 0, 0, 0, 0);
                 }
-                mma_commit(bar(kBarPFree));
-                mma_commit(bar(kBarEmpty0 + (pn % kStages)));
-                mma_commit(bar(kBarOFull));
+                fence_proxy_async_smem();
             }
             __syncwarp();
-            ++s_cnt;
+            // S(g) reuses the S columns: the softmax warps must have read S(g-1).
+            if (g > 0 && !mbar_wait(bar(kBarSFree), (g - 1) & 1)) { ok = false; break; }
+            tc_fence_after();
+            MLA_TRACE_POINT(2, g);
+            if (lane == 0) {
+                // S = Qhat_half . C_half^T: 4 latent chunks x 4 K-steps, then 2 RoPE K-steps
+                for (int c = 0; c < 4; ++c)
+                    for (int k = 0; k < 4; ++k) {
+                        const uint64_t bd = smem_desc(tile + c * (kNk * 128) + 32 * k, 16, 1024, kSw128);
+                        mma_f16_ts(tmem + kTmemS, tmem + kTmemQ + 8 * (4 * c + k), bd, idS, (c | k) ? 1u : 0u);
+                    }
+                for (int k = 0; k < 2; ++k) {
+                    const uint64_t bd = smem_desc(tile + 4 * (kNk * 128) + 32 * k, 16, 512, kSw64);
+                    mma_f16_ts(tmem + kTmemS, tmem + kTmemQ + 128 + 8 * k, bd, idS, 1u);
+                }
+                mma_commit(bar(kBarSFull));
+            }
+            __syncwarp();
+            MLA_TRACE_POINT(3, g);
+            if (g > 0) {
+                if (!mbar_wait(bar(kBarPFull), (g - 1) & 1)) { ok = false; break; }
+                if (prev_first && prev_seg > 0 && !mbar_wait(bar(kBarOFree), (prev_seg - 1) & 1)) { ok = false; break; }
+                tc_fence_after();
+                MLA_TRACE_POINT(4, g - 1);
+                if (lane == 0) issue_O(g - 1, prev_first, prev_last);
+                __syncwarp();
+                MLA_TRACE_POINT(5, g - 1);
+            }
+            prev_first = w.first();
+            prev_last = w.last();
+            prev_seg = w.seg;
+        }
+        if (ok && !*abort_flag && g > 0) {
+            if (!mbar_wait(bar(kBarPFull), (g - 1) & 1)) ok = false;
+            else if (prev_first && prev_seg > 0 && !mbar_wait(bar(kBarOFree), (prev_seg - 1) & 1)) ok = false;
+            else {
+                tc_fence_after();
+                if (lane == 0) issue_O(g - 1, prev_first, prev_last);
+                __syncwarp();
+            }
         }
         if (!ok) *abort_flag = 1;
     } else {
-        // ======================================================== softmax warps 2..5
+        // ======================================================== softmax warps 2..5 (row r = head r)
+        // Software pipeline: iteration g publishes the partial scores of tile
+        // g+1 before it runs the softmax of tile g, so the exchange with the
+        // peer overlaps a whole iteration.  Each CTA writes its fp16 partial
+        // scores into its own shared memory and the peer pulls them with
+        // ld.shared::cluster; one remote arrive per warp signals "published"
+        // and one signals "read".
         const int quarter = warp & 3;
-        const int r = quarter * 32 + lane;  // head / TMEM lane
+        const int r = quarter * 32 + lane;
         const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
         const uint32_t x_local = base + kOffX;
         const uint32_t x_peer = mapa(x_local, peer);
-        const uint32_t xfull_peer = mapa(bar(kBarXFull), peer);
-        const uint32_t xempty_peer = mapa(bar(kBarXEmpty), peer);
+        const uint32_t xready_peer0 = mapa(bar(kBarXReady0), peer);
+        const uint32_t xread_peer0 = mapa(bar(kBarXRead0), peer);
         const float sl2 = args.scale_log2;
-        int n = 0, s_cnt = 0;
         bool ok = true;
-        while (ok && !*abort_flag && it.next(seq, k0, k1, whole)) {
-            const int T_b = args.seqlens[seq];
-            const int n_keys = T_b - q_len + 1 + qi;  // query qi attends to keys 0..n_keys-1
-            float m_used = -CUDART_INF_F, l_sum = 0.f;
-            for (int t = k0; t < k1; ++t, ++n) {
-                float s[kNk];
-                // ---- partial S of this half
-                if (!mbar_wait(bar(kBarSFull), n & 1)) { ok = false; break; }
-                tc_fence_after();
-                {
-                    uint32_t v[32];
-                    tmem_ld32(tmem + lane_addr + kTmemS, v);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) s[j] = __uint_as_float(v[j]);
-                    tmem_ld32(tmem + lane_addr + kTmemS + 32, v);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) s[32 + j] = __uint_as_float(v[j]);
-                }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(kBarSFree));
-                // ---- swap partial S with the peer half
-                if (n > 0 && !mbar_wait_cluster(bar(kBarXEmpty), (n - 1) & 1)) { ok = false; break; }
-                if (threadIdx.x == 64) mbar_arrive_expect_tx(bar(kBarXFull), kXBytes);
-#pragma unroll
-                for (int ch = 0; ch < 16; ++ch) {
-                    const uint32_t off = (uint32_t)(r * 256 + ((ch ^ (r & 15)) << 4));
-                    st_async_v4(x_peer + off, s[4 * ch], s[4 * ch + 1], s[4 * ch + 2], s[4 * ch + 3], xfull_peer);
-                }
-                if (!mbar_wait_cluster(bar(kBarXFull), n & 1)) { ok = false; break; }
-                // Both halves add (own + peer) in the same order: half 0 first.
-#pragma unroll
-                for (int ch = 0; ch < 16; ++ch) {
-                    float a, b2, c, d;
-                    ld_shared_v4f(x_local + (uint32_t)(r * 256 + ((ch ^ (r & 15)) << 4)), a, b2, c, d);
-                    if (half == 0) {
-                        s[4 * ch] += a; s[4 * ch + 1] += b2; s[4 * ch + 2] += c; s[4 * ch + 3] += d;
-                    } else {
-                        s[4 * ch] = a + s[4 * ch]; s[4 * ch + 1] = b2 + s[4 * ch + 1];
-                        s[4 * ch + 2] = c + s[4 * ch + 2]; s[4 * ch + 3] = d + s[4 * ch + 3];
-                    }
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive_remote(xempty_peer);
-                // ---- online softmax (base 2), lazy rescale of O
-                const int key0 = t * kNk;
-                float mx = -CUDART_INF_F;
-#pragma unroll
-                for (int j = 0; j < kNk; ++j) {
-                    s[j] = (key0 + j < n_keys) ? s[j] * sl2 : -CUDART_INF_F;
-                    mx = fmaxf(mx, s[j]);
-                }
-                const bool first = (t == k0);
-                const bool grow = mx > m_used + 8.0f;  // rescale only when the max grows by > 2^8
-                // P(n) overwrites P(n-1) and a rescale touches O: wait for O += P(n-1) C(n-1).
-                if (n > 0 && !mbar_wait(bar(kBarPFree), (n - 1) & 1)) { ok = false; break; }
-                tc_fence_after();
-                if (grow) {
-                    if (!first) {
-                        const float f = ex2(m_used - mx);
-                        l_sum *= f;
-#pragma unroll 1
-                        for (int c0 = 0; c0 < kHalfLat; c0 += 32) {
-                            uint32_t v[32];
-                            tmem_ld32(tmem + lane_addr + kTmemO + c0, v);
-                            tmem_wait_ld();
-#pragma unroll
-                            for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * f);
-                            tmem_st32(tmem + lane_addr + kTmemO + c0, v);
-                        }
-                        tmem_wait_st();
-                    }
-                    m_used = mx;
-                }
-                const float mb = (m_used == -CUDART_INF_F) ? 0.f : m_used;
-                float rs = 0.f;
-                const uint32_t prow = base + kOffP;
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    float p0 = ex2(s[8 * k + 0] - mb), p1 = ex2(s[8 * k + 1] - mb);
-                    float p2 = ex2(s[8 * k + 2] - mb), p3 = ex2(s[8 * k + 3] - mb);
-                    float p4 = ex2(s[8 * k + 4] - mb), p5 = ex2(s[8 * k + 5] - mb);
-                    float p6 = ex2(s[8 * k + 6] - mb), p7 = ex2(s[8 * k + 7] - mb);
-                    rs += ((p0 + p1) + (p2 + p3)) + ((p4 + p5) + (p6 + p7));
-                    st_shared_v4(prow + sw128_off(r, k), pack_bf16(p0, p1), pack_bf16(p2, p3), pack_bf16(p4, p5),
-                                 pack_bf16(p6, p7));
-                }
-                l_sum += rs;
-                fence_proxy_async_smem();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(kBarPFull));
-            }
-            if (!ok) break;
-            // ---- epilogue of this segment
-            if (!mbar_wait(bar(kBarOFull), s_cnt & 1)) { ok = false; break; }
-            tc_fence_after();
-            const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
+
+        // this half of Q-hat row r -> TMEM columns kTmemQ.. (144 columns)
+        auto load_q = [&](int seq) {
             const int u = seq * q_len + qi;
-            if (whole) {
-                __nv_bfloat16* dst = args.o_lat + ((size_t)u * kHeads + r) * kLat + half * kHalfLat;
+            const uint4* src = reinterpret_cast<const uint4*>(args.q_hat + ((size_t)u * kHeads + r) * kRow);
 #pragma unroll 1
-                for (int c0 = 0; c0 < kHalfLat; c0 += 32) {
-                    uint32_t v[32];
-                    tmem_ld32(tmem + lane_addr + kTmemO + c0, v);
-                    tmem_wait_ld();
+            for (int c = 0; c < 4; ++c) {
+                uint32_t v[32];
 #pragma unroll
-                    for (int j = 0; j < 32; j += 8) {
-                        uint4 w;
-                        w.x = pack_bf16(__uint_as_float(v[j]) * inv, __uint_as_float(v[j + 1]) * inv);
-                        w.y = pack_bf16(__uint_as_float(v[j + 2]) * inv, __uint_as_float(v[j + 3]) * inv);
-                        w.z = pack_bf16(__uint_as_float(v[j + 4]) * inv, __uint_as_float(v[j + 5]) * inv);
-                        w.w = pack_bf16(__uint_as_float(v[j + 6]) * inv, __uint_as_float(v[j + 7]) * inv);
-                        *reinterpret_cast<uint4*>(dst + c0 + j) = w;
-                    }
+                for (int j = 0; j < 8; ++j) {
+                    const uint4 x = __ldg(src + half * 32 + c * 8 + j);
+                    v[4 * j] = x.x; v[4 * j + 1] = x.y; v[4 * j + 2] = x.z; v[4 * j + 3] = x.w;
                 }
-            } else {
-                const int slot = cl + seq;
-                float* dst = args.part_o + (((size_t)slot * q_len + qi) * kHeads + r) * kLat + half * kHalfLat;
-#pragma unroll 1
-                for (int c0 = 0; c0 < kHalfLat; c0 += 32) {
-                    uint32_t v[32];
-                    tmem_ld32(tmem + lane_addr + kTmemO + c0, v);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int j = 0; j < 32; j += 4) {
-                        float4 w = make_float4(__uint_as_float(v[j]) * inv, __uint_as_float(v[j + 1]) * inv,
-                                               __uint_as_float(v[j + 2]) * inv, __uint_as_float(v[j + 3]) * inv);
-                        *reinterpret_cast<float4*>(dst + c0 + j) = w;
-                    }
-                }
-                if (half == 0)
-                    args.part_lse[((size_t)slot * q_len + qi) * kHeads + r] =
-                        l_sum > 0.f ? m_used + __log2f(l_sum) : -CUDART_INF_F;
+                tmem_st32(tmem + lane_addr + kTmemQ + 32 * c, v);
             }
+            uint32_t v[16];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const uint4 x = __ldg(src + 64 + half * 4 + j);
+                v[4 * j] = x.x; v[4 * j + 1] = x.y; v[4 * j + 2] = x.z; v[4 * j + 3] = x.w;
+            }
+            tmem_st16(tmem + lane_addr + kTmemQ + 128, v);
+            tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(kBarOFree));
-            ++s_cnt;
+            if (lane == 0) mbar_arrive(bar(kBarQFull));
+        };
+        // partial S(g) out of TMEM, scaled to log2 units, published as fp16 in
+        // our buffer g & 1; own copy kept (rounded the same way) in `mine`.
+        auto fetch_send = [&](int g, uint32_t (&mine)[32]) -> bool {
+            if (!mbar_wait(bar(kBarSFull), g & 1)) return false;
+            tc_fence_after();
+            MLA_TRACE_POINT(7, g);
+            uint32_t v[32], v2[32];
+            tmem_ld32(tmem + lane_addr + kTmemS, v);
+            tmem_ld32(tmem + lane_addr + kTmemS + 32, v2);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(kBarSFree));
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                mine[j] = pack_f16(__uint_as_float(v[2 * j]) * sl2, __uint_as_float(v[2 * j + 1]) * sl2);
+                mine[16 + j] = pack_f16(__uint_as_float(v2[2 * j]) * sl2, __uint_as_float(v2[2 * j + 1]) * sl2);
+            }
+            const int b = g & 1;
+            // the peer must have finished reading what we published in this buffer two tiles ago
+            if (g >= 2 && !mbar_wait_cluster(bar(kBarXRead0 + b), ((g - 2) >> 1) & 1)) return false;
+            MLA_TRACE_POINT(8, g);
+            const uint32_t dst = x_local + b * kXBytes + r * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                st_shared_v4(dst + ((c ^ (r & 7)) << 4), mine[4 * c], mine[4 * c + 1], mine[4 * c + 2], mine[4 * c + 3]);
+            fence_acq_rel_cluster();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote(xready_peer0 + 8 * b);
+            MLA_TRACE_POINT(9, g);
+            return true;
+        };
+
+        TileWalk cur, nxt;
+        cur.init(args.plan, cl);
+        nxt = cur;
+        uint32_t mine_cur[32], mine_nxt[32];
+        if (cur.valid) {
+            load_q(cur.seq);
+            ok = fetch_send(0, mine_cur);
+            nxt.advance();
+        }
+        float m_used = -CUDART_INF_F, l_sum = 0.f;
+        int g = 0;
+        for (; cur.valid && ok && !*abort_flag; ++g) {
+            if (nxt.valid) {
+                if (nxt.seg != cur.seg) load_q(nxt.seq);  // S(g) was read: Q-hat columns are free
+                if (!fetch_send(g + 1, mine_nxt)) { ok = false; break; }
+            }
+            // ---- pull the peer's partial S(g) and add it (half 0's part first)
+            const int b = g & 1;
+            if (!mbar_wait_cluster(bar(kBarXReady0 + b), (g >> 1) & 1)) { ok = false; break; }
+            MLA_TRACE_POINT(10, g);
+            float s[kNk];
+            const uint32_t src = x_peer + b * kXBytes + r * 128;
+            uint32_t xs[32];
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                ld_cluster_v4u(src + ((c ^ (r & 7)) << 4), xs[4 * c], xs[4 * c + 1], xs[4 * c + 2], xs[4 * c + 3]);
+#pragma unroll
+            for (int q = 0; q < 32; ++q) {
+                const float2 o = unpack_f16(xs[q]);
+                const float2 m = unpack_f16(mine_cur[q]);
+                s[2 * q] = half == 0 ? m.x + o.x : o.x + m.x;
+                s[2 * q + 1] = half == 0 ? m.y + o.y : o.y + m.y;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote(xread_peer0 + 8 * b);
+            // ---- online softmax in base 2 with lazy rescaling of O
+            const int T_b = args.seqlens[cur.seq];
+            const int n_keys = T_b - q_len + 1 + qi;  // query qi attends to keys 0..n_keys-1
+            const int key0 = cur.t * kNk;
+            if (key0 + kNk > n_keys) {
+#pragma unroll
+                for (int j = 0; j < kNk; ++j)
+                    if (key0 + j >= n_keys) s[j] = -CUDART_INF_F;
+            }
+            float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+#pragma unroll
+            for (int j = 4; j < kNk; j += 4) {
+                mx0 = fmaxf(mx0, s[j]); mx1 = fmaxf(mx1, s[j + 1]);
+                mx2 = fmaxf(mx2, s[j + 2]); mx3 = fmaxf(mx3, s[j + 3]);
+            }
+            const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+            const bool first = cur.first();
+            const bool grow = mx > m_used + 8.0f;  // rescale only when the max grows by > 2^8
+            const float mb_new = grow ? mx : m_used;
+            const float mb = (mb_new == -CUDART_INF_F) ? 0.f : mb_new;
+            uint32_t pk[32];
+            float rs0 = 0.f, rs1 = 0.f;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const float p0 = ex2(s[2 * j] - mb), p1 = ex2(s[2 * j + 1] - mb);
+                rs0 += p0;
+                rs1 += p1;
+                pk[j] = pack_bf16(p0, p1);
+            }
+            MLA_TRACE_POINT(11, g);
+            // P(g) overwrites P(g-1) and a rescale touches O: wait for O += P(g-1) C(g-1).
+            if (g > 0 && !mbar_wait(bar(kBarPFree), (g - 1) & 1)) { ok = false; break; }
+            tc_fence_after();
+            MLA_TRACE_POINT(12, g);
+            if (grow) {
+                if (!first) {
+                    const float f = ex2(m_used - mx);
+                    l_sum *= f;
+#pragma unroll 1
+                    for (int c0 = 0; c0 < kHalfLat; c0 += 32) {
+                        uint32_t v[32];
+                        tmem_ld32(tmem + lane_addr + kTmemO + c0, v);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * f);
+                        tmem_st32(tmem + lane_addr + kTmemO + c0, v);
+                    }
+                }
+                m_used = mx;
+            }
+            l_sum += rs0 + rs1;
+            tmem_st32(tmem + lane_addr + kTmemP, pk);
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(kBarPFull));
+            MLA_TRACE_POINT(13, g);
+            // ---- epilogue at the end of a piece
+            if (cur.last()) {
+                if (!mbar_wait(bar(kBarOFull), cur.seg & 1)) { ok = false; break; }
+                tc_fence_after();
+                const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
+                const int u = cur.seq * q_len + qi;
+                if (cur.whole) {
+                    __nv_bfloat16* dst = args.o_lat + ((size_t)u * kHeads + r) * kLat + half * kHalfLat;
+#pragma unroll 1
+                    for (int c0 = 0; c0 < kHalfLat; c0 += 32) {
+                        uint32_t v[32];
+                        tmem_ld32(tmem + lane_addr + kTmemO + c0, v);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 32; j += 8) {
+                            uint4 w;
+                            w.x = pack_bf16(__uint_as_float(v[j]) * inv, __uint_as_float(v[j + 1]) * inv);
+                            w.y = pack_bf16(__uint_as_float(v[j + 2]) * inv, __uint_as_float(v[j + 3]) * inv);
+                            w.z = pack_bf16(__uint_as_float(v[j + 4]) * inv, __uint_as_float(v[j + 5]) * inv);
+                            w.w = pack_bf16(__uint_as_float(v[j + 6]) * inv, __uint_as_float(v[j + 7]) * inv);
+                            *reinterpret_cast<uint4*>(dst + c0 + j) = w;
+                        }
+                    }
+                } else {
+                    const int slot = cl + cur.seq;
+                    float* dst = args.part_o + (((size_t)slot * q_len + qi) * kHeads + r) * kLat + half * kHalfLat;
+#pragma unroll 1
+                    for (int c0 = 0; c0 < kHalfLat; c0 += 32) {
+                        uint32_t v[32];
+                        tmem_ld32(tmem + lane_addr + kTmemO + c0, v);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 32; j += 4) {
+                            float4 w = make_float4(__uint_as_float(v[j]) * inv, __uint_as_float(v[j + 1]) * inv,
+                                                   __uint_as_float(v[j + 2]) * inv, __uint_as_float(v[j + 3]) * inv);
+                            *reinterpret_cast<float4*>(dst + c0 + j) = w;
+                        }
+                    }
+                    if (half == 0)
+                        args.part_lse[((size_t)slot * q_len + qi) * kHeads + r] =
+                            l_sum > 0.f ? m_used + __log2f(l_sum) : -CUDART_INF_F;
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(kBarOFree));
+                m_used = -CUDART_INF_F;
+                l_sum = 0.f;
+            }
+            // advance the pipeline
+#pragma unroll
+            for (int j = 0; j < 32; ++j) mine_cur[j] = mine_nxt[j];
+            cur = nxt;
+            if (nxt.valid) nxt.advance();
         }
         if (!ok) *abort_flag = 1;
     }
@@ -493,7 +579,7 @@ __global__ void __launch_bounds__(kAttThreads, 1)
     tc_fence_before();
     __syncthreads();
     if (warp == 1) tmem_dealloc(tmem, kTmemCols);
-    // The peer may still read our barriers / write our X buffer until it is done.
+    // The peer may still read our barriers / write our X buffers until it is done.
     cluster_sync();
 }
 
