@@ -196,8 +196,13 @@ def run_ours(args, rank, world, local_rank):
     s = torch.cuda.Stream(device)
     s.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(s):
-        for _ in range(2):
-            step(stream=s)
+        step(stream=s)
+    torch.cuda.current_stream().wait_stream(s)
+    status = lib.device_status()
+    if status:
+        raise RuntimeError(f"the first decode step reported device status {status}; not timing it")
+    with torch.cuda.stream(s):
+        step(stream=s)
     torch.cuda.current_stream().wait_stream(s)
     torch.cuda.synchronize()
     path = lib.last_path()

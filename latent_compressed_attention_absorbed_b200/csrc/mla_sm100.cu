@@ -218,10 +218,9 @@ cudaError_t sm100_attend(const Problem& p, const void* q_hat, const CacheView& c
     if (ws_bytes < need) return cudaErrorInvalidValue;
     char* ws = static_cast<char*>(workspace);
     Plan* plan = reinterpret_cast<Plan*>(ws);
-    CUtensorMap mCL, mCR;
+    CUtensorMap mC;
     const uint64_t sb = (uint64_t)cache.stride_b * 2, stt = (uint64_t)cache.stride_t * 2;
-    if (!make_map(&mCL, cache.data, kRow, cache.T_max, p.B, stt, sb, 64, kNk, 1, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&mCR, cache.data, kRow, cache.T_max, p.B, stt, sb, 32, kNk, 1, CU_TENSOR_MAP_SWIZZLE_64B))
+    if (!make_map(&mC, cache.data, kRow, cache.T_max, p.B, stt, sb, 64, kNk, 1, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
 
     const int ovh = overhead_tiles < 0 ? 2 : overhead_tiles;
@@ -258,7 +257,7 @@ cudaError_t sm100_attend(const Problem& p, const void* q_hat, const CacheView& c
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     if (events) events->record(MLA_EV_ATTEND_BEGIN, st);
-    e = cudaLaunchKernelEx(&cfg, mla_attend_kernel, mCL, mCR, a);
+    e = cudaLaunchKernelEx(&cfg, mla_attend_kernel, mC, a);
     if (e != cudaSuccess) return e;
     if (events) events->record(MLA_EV_ATTEND_END, st);
 

@@ -10,16 +10,18 @@
 // aggregate sum_j p_j c_KV,j before W_UV; m.lsln.cn section 2.1: softmax over
 // the whole history.)
 //
-// Work split.  The fp32 accumulator of all 128 heads x 512 latent columns
-// would fill the whole 512-column TMEM, leaving no room for S.  A cluster of
-// two CTAs therefore splits the 576-wide cache row: CTA "half" 0 takes latent
-// columns 0..255 and RoPE columns 0..31, CTA 1 takes 256..511 and 32..63.
-// Each computes a partial S over its 288 columns, the pair swaps partial S
-// through distributed shared memory (st.async completing on the peer's
-// mbarrier), both add the two halves in the same order, run the same
-// softmax, and each accumulates its 256 latent columns of O in TMEM.  The
-// cache is read from HBM exactly once.  With q_len query tokens the cluster
-// holds q_len such pairs that stream the same cache tiles together.
+// Work split.  A CTA owns 64 of the 128 heads of one query token and streams
+// full 576-wide cache tiles; the two CTAs of a head pair (and the q_len
+// token groups) form one cluster so that they run together and each tile is
+// read from HBM once and served to the others from L2.  Nothing is
+// exchanged between CTAs.  Per CTA the fp32 accumulator is 64 heads x 512
+// latent columns: latent 0..255 lives in TMEM lanes 0..15 of each 32-lane
+// subpartition and latent 256..511 in lanes 16..31, both in columns 0..255
+// (M = 64 MMAs address either lane half).  Scores are split the same way:
+// the lower lane half accumulates S over latent 0..255 + RoPE 0..31, the
+// upper half over latent 256..511 + RoPE 32..63, and the two partial sums
+// of a row are added with one warp shuffle (lanes t and t+16 hold the same
+// head).
 //
 // Scheduling (split-KV).  Sequences are cut into 64-key tiles; the clusters
 // divide the concatenated tile list into equal contiguous ranges (a fixed
@@ -29,9 +31,10 @@
 // head, merged by the combine kernel.
 //
 // Roles per CTA (192 threads): warp 0 TMA producer, warp 1 TMEM owner and
-// MMA issuer, warps 2..5 softmax (warp w owns TMEM lanes 32*(w%4)..+31, i.e.
-// heads).  Every wait is bounded; on expiry the kernel flags
-// MLA_STATUS_TIMEOUT, stops issuing work and tears down normally.
+// MMA issuer, warps 2..5 softmax (warp w reads TMEM subpartition w%4: heads
+// 16*(w%4)..+15 in both lane halves).  Every wait is bounded; on expiry the
+// kernel flags MLA_STATUS_TIMEOUT, stops issuing work and tears down
+// normally.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -43,31 +46,30 @@ namespace mla {
 namespace sm100 {
 
 constexpr int kNk = 64;          // keys per tile
-constexpr int kHeads = 128;      // M
+constexpr int kHeads = 128;      // heads of a token
+constexpr int kRowsCta = 64;     // heads per CTA (M of every MMA)
 constexpr int kLat = 512;        // d_c
 constexpr int kRope = 64;        // d_r
 constexpr int kRow = kLat + kRope;
 constexpr int kHalfLat = 256;
 constexpr int kHalfRope = 32;
 
-// Shared-memory map (offsets from a 1024-aligned base): a ring of cache
-// tiles (each: 4 SW128 chunks of 64 keys x 64 latent columns, then one SW64
-// chunk of 64 keys x 32 RoPE columns) and two buffers in which this CTA
-// publishes its partial scores for the peer to read.  Q-hat and P live in
-// tensor memory.
-constexpr int kTileBytes = kNk * 128 * 4 + kNk * 64;       // 36864
-constexpr int kStages = 5;
-constexpr int kXBytes = kHeads * kNk * 2;                  // 128 x 64 fp16 partial scores
+// Shared-memory map (offsets from a 1024-aligned base): a ring of full cache
+// tiles, each 9 SW128 chunks of 64 keys x 64 columns (8 latent, 1 RoPE).
+constexpr int kChunk = kNk * 128;                          // 8192
+constexpr int kTileBytes = 9 * kChunk;                     // 73728
+constexpr int kStages = 3;
 constexpr int kOffTiles = 0;
-constexpr int kOffX = kOffTiles + kStages * kTileBytes;    // two publish buffers
-constexpr int kOffBars = kOffX + 2 * kXBytes;
+constexpr int kOffBars = kOffTiles + kStages * kTileBytes;
 constexpr int kAttSmem = kOffBars + 256 + 1024;
-// Tensor-memory map (columns of 32 bits, 128 lanes = heads).
+// Tensor-memory map: columns of 32 bits; lane half 0 = lanes 0..15 of each
+// subpartition, lane half 1 = lanes 16..31 (address lane field + 16).
 constexpr int kTmemCols = 512;
-constexpr int kTmemO = 0;      // O: 256 fp32 latent columns of this half
-constexpr int kTmemS = 256;    // S: 64 fp32 scores (partial, this half's 288 columns)
-constexpr int kTmemP = 320;    // P: 64 bf16 probabilities, two per column
-constexpr int kTmemQ = 352;    // Q-hat half: 256 latent + 32 RoPE bf16, two per column (144 columns)
+constexpr uint32_t kLaneHalf1 = 16u << 16;
+constexpr int kTmemO = 0;      // O: half 0 latent 0..255, half 1 latent 256..511 (256 columns)
+constexpr int kTmemS = 256;    // S: half 0 partial over K-half a, half 1 over K-half b (64 columns)
+constexpr int kTmemP = 320;    // P: 64 bf16 probabilities, two per column, copied in both halves
+constexpr int kTmemQ = 352;    // Q-hat: half 0 latent 0..255 + RoPE 0..31, half 1 the rest (144 columns)
 constexpr int kAttThreads = 192;
 
 // Barrier indices (8 bytes each) inside the barrier block.
@@ -75,17 +77,12 @@ enum {
     kBarFull0 = 0,
     kBarEmpty0 = kBarFull0 + kStages,
     kBarQFull = kBarEmpty0 + kStages,
-    kBarQEmpty,
     kBarSFull,
     kBarSFree,
     kBarPFull,
     kBarPFree,
     kBarOFull,
     kBarOFree,
-    kBarXReady0,  // peer has published its partial S in its buffer 0 / 1
-    kBarXReady1,
-    kBarXRead0,   // peer has finished reading our buffer 0 / 1
-    kBarXRead1,
     kNumBars
 };
 
@@ -195,8 +192,7 @@ struct AttendArgs {
 };
 
 __global__ void __launch_bounds__(kAttThreads, 1)
-    mla_attend_kernel(const __grid_constant__ CUtensorMap mapCacheLat, const __grid_constant__ CUtensorMap mapCacheRope,
-                      AttendArgs args) {
+    mla_attend_kernel(const __grid_constant__ CUtensorMap mapCache, AttendArgs args) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -207,9 +203,8 @@ __global__ void __launch_bounds__(kAttThreads, 1)
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const uint32_t crank = cluster_ctarank();
-    const int half = crank & 1;
-    const int qi = crank >> 1;
-    const uint32_t peer = crank ^ 1u;
+    const int hpart = crank & 1;       // heads 64*hpart .. +63
+    const int qi = crank >> 1;         // query token of this CTA
     const int cl = (int)cluster_id_x();
     const int q_len = args.q_len;
 
@@ -219,29 +214,22 @@ __global__ void __launch_bounds__(kAttThreads, 1)
             mbar_init(bar(kBarEmpty0 + s), 1);
         }
         mbar_init(bar(kBarQFull), 4);
-        mbar_init(bar(kBarQEmpty), 1);
         mbar_init(bar(kBarSFull), 1);
         mbar_init(bar(kBarSFree), 4);
         mbar_init(bar(kBarPFull), 4);
         mbar_init(bar(kBarPFree), 1);
         mbar_init(bar(kBarOFull), 1);
         mbar_init(bar(kBarOFree), 4);
-        mbar_init(bar(kBarXReady0), 4);
-        mbar_init(bar(kBarXReady1), 4);
-        mbar_init(bar(kBarXRead0), 4);
-        mbar_init(bar(kBarXRead1), 4);
         *abort_flag = 0;
         fence_mbar_init();
-        prefetch_tensormap(&mapCacheLat);
-        prefetch_tensormap(&mapCacheRope);
+        prefetch_tensormap(&mapCache);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
     }
     tc_fence_before();
-    // Peer barriers must be initialised before any remote arrive / st.async.
-    cluster_sync();
+    __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(base_ptr + kOffBars + 8 * kNumBars);
 
@@ -258,25 +246,25 @@ __global__ void __launch_bounds__(kAttThreads, 1)
                 }
                 const uint32_t dst = base + kOffTiles + st * kTileBytes;
                 mbar_arrive_expect_tx(bar(kBarFull0 + st), kTileBytes);
-                for (int c = 0; c < 4; ++c)
-                    tma_load_3d(dst + c * (kNk * 128), &mapCacheLat, bar(kBarFull0 + st), half * kHalfLat + 64 * c,
-                                w.t * kNk, w.seq);
-                tma_load_3d(dst + 4 * (kNk * 128), &mapCacheRope, bar(kBarFull0 + st), kLat + half * kHalfRope,
-                            w.t * kNk, w.seq);
+                for (int c = 0; c < 9; ++c)
+                    tma_load_3d(dst + c * kChunk, &mapCache, bar(kBarFull0 + st), 64 * c, w.t * kNk, w.seq);
                 MLA_TRACE_POINT(0, n);
             }
         }
     } else if (warp == 1) {
         // ======================================================== MMA issuer (whole warp waits, lane 0 issues)
-        constexpr uint32_t idS = idesc_bf16_f32(128, kNk, false, false);
-        constexpr uint32_t idO = idesc_bf16_f32(128, kHalfLat, false, true);
+        constexpr uint32_t idS = idesc_bf16_f32(kRowsCta, kNk, false, false);
+        constexpr uint32_t idO = idesc_bf16_f32(kRowsCta, kHalfLat, false, true);
         bool ok = true;
-        // O(g) += P(g) . C(g); its first K-step overwrites O at the start of a piece.
+        // O(g) += P(g) . C(g) for both latent halves; the first K-step overwrites O at the start of a piece.
         auto issue_O = [&](int g, bool first_in_seg, bool last_in_seg) {
-            const uint32_t ptile = base + kOffTiles + (g % kStages) * kTileBytes;
+            const uint32_t tile = base + kOffTiles + (g % kStages) * kTileBytes;
             for (int k = 0; k < 4; ++k) {
-                const uint64_t bd = smem_desc(ptile + 2048 * k, kNk * 128, 1024, kSw128);
-                mma_f16_ts(tmem + kTmemO, tmem + kTmemP + 8 * k, bd, idO, (!first_in_seg || k > 0) ? 1u : 0u);
+                const uint32_t acc = (!first_in_seg || k > 0) ? 1u : 0u;
+                mma_f16_ts(tmem + kTmemO, tmem + kTmemP + 8 * k, smem_desc(tile + 2048 * k, kChunk, 1024, kSw128),
+                           idO, acc);
+                mma_f16_ts(tmem + kLaneHalf1 + kTmemO, tmem + kLaneHalf1 + kTmemP + 8 * k,
+                           smem_desc(tile + 4 * kChunk + 2048 * k, kChunk, 1024, kSw128), idO, acc);
             }
             mma_commit(bar(kBarPFree));
             mma_commit(bar(kBarEmpty0 + (g % kStages)));
@@ -284,10 +272,25 @@ __global__ void __launch_bounds__(kAttThreads, 1)
         };
         TileWalk w;
         w.init(args.plan, cl);
-        bool prev_first = false, prev_last = false;
+        bool prev_first = false, prev_last = false, prev_pending = false;
         int prev_seg = 0;
         int g = 0;
+        // O(g-1) normally follows S(g) so that S(g) overlaps the softmax of
+        // tile g-1; at the end of a piece it goes first, because the softmax
+        // warps load the next piece's Q-hat only after that piece's epilogue.
+        auto finish_prev = [&]() -> bool {
+            if (!mbar_wait(bar(kBarPFull), (g - 1) & 1)) return false;
+            if (prev_first && prev_seg > 0 && !mbar_wait(bar(kBarOFree), (prev_seg - 1) & 1)) return false;
+            tc_fence_after();
+            MLA_TRACE_POINT(4, g - 1);
+            if (lane == 0) issue_O(g - 1, prev_first, prev_last);
+            __syncwarp();
+            MLA_TRACE_POINT(5, g - 1);
+            prev_pending = false;
+            return true;
+        };
         for (; w.valid && ok && !*abort_flag; ++g, w.advance()) {
+            if (prev_pending && prev_last && !finish_prev()) { ok = false; break; }
             const int T_b = args.seqlens[w.seq];
             if (w.first() && !mbar_wait(bar(kBarQFull), w.seg & 1)) { ok = false; break; }
             const int st = g % kStages;
@@ -299,11 +302,8 @@ __global__ void __launch_bounds__(kAttThreads, 1)
                 // Rows at or beyond T_b hold no cached token: zero them so that
                 // masked (p = 0) rows cannot inject NaN/Inf into P.C.
                 const int r0 = valid < 0 ? 0 : valid;
-                for (int r = r0 + (lane >> 3); r < kNk; r += 4) {
-                    for (int c = 0; c < 4; ++c)
-                        st_shared_v4(tile + c * (kNk * 128) + r * 128 + (lane & 7) * 16, 0, 0, 0, 0);
-                    if ((lane & 7) < 4) st_shared_v4(tile + 4 * (kNk * 128) + r * 64 + (lane & 7) * 16, 0, 0, 0, 0);
-                }
+                for (int r = r0 + (lane >> 3); r < kNk; r += 4)
+                    for (int c = 0; c < 9; ++c) st_shared_v4(tile + c * kChunk + r * 128 + (lane & 7) * 16, 0, 0, 0, 0);
                 fence_proxy_async_smem();
             }
             __syncwarp();
@@ -312,183 +312,127 @@ __global__ void __launch_bounds__(kAttThreads, 1)
             tc_fence_after();
             MLA_TRACE_POINT(2, g);
             if (lane == 0) {
-                // S = Qhat_half . C_half^T: 4 latent chunks x 4 K-steps, then 2 RoPE K-steps
-                for (int c = 0; c < 4; ++c)
-                    for (int k = 0; k < 4; ++k) {
-                        const uint64_t bd = smem_desc(tile + c * (kNk * 128) + 32 * k, 16, 1024, kSw128);
-                        mma_f16_ts(tmem + kTmemS, tmem + kTmemQ + 8 * (4 * c + k), bd, idS, (c | k) ? 1u : 0u);
-                    }
-                for (int k = 0; k < 2; ++k) {
-                    const uint64_t bd = smem_desc(tile + 4 * (kNk * 128) + 32 * k, 16, 512, kSw64);
-                    mma_f16_ts(tmem + kTmemS, tmem + kTmemQ + 128 + 8 * k, bd, idS, 1u);
+                // half a: latent chunks 0..3 then RoPE columns 0..31; half b: chunks 4..7 then RoPE 32..63
+                for (int kk = 0; kk < 18; ++kk) {
+                    const int ca = kk < 16 ? kk / 4 : 8, cb = kk < 16 ? 4 + kk / 4 : 8;
+                    const int oa = kk < 16 ? 32 * (kk % 4) : 32 * (kk - 16);
+                    const int ob = kk < 16 ? 32 * (kk % 4) : 64 + 32 * (kk - 16);
+                    mma_f16_ts(tmem + kTmemS, tmem + kTmemQ + 8 * kk,
+                               smem_desc(tile + ca * kChunk + oa, 16, 1024, kSw128), idS, kk ? 1u : 0u);
+                    mma_f16_ts(tmem + kLaneHalf1 + kTmemS, tmem + kLaneHalf1 + kTmemQ + 8 * kk,
+                               smem_desc(tile + cb * kChunk + ob, 16, 1024, kSw128), idS, kk ? 1u : 0u);
                 }
                 mma_commit(bar(kBarSFull));
             }
             __syncwarp();
             MLA_TRACE_POINT(3, g);
-            if (g > 0) {
-                if (!mbar_wait(bar(kBarPFull), (g - 1) & 1)) { ok = false; break; }
-                if (prev_first && prev_seg > 0 && !mbar_wait(bar(kBarOFree), (prev_seg - 1) & 1)) { ok = false; break; }
-                tc_fence_after();
-                MLA_TRACE_POINT(4, g - 1);
-                if (lane == 0) issue_O(g - 1, prev_first, prev_last);
-                __syncwarp();
-                MLA_TRACE_POINT(5, g - 1);
-            }
+            if (prev_pending && !finish_prev()) { ok = false; break; }
             prev_first = w.first();
             prev_last = w.last();
             prev_seg = w.seg;
+            prev_pending = true;
         }
-        if (ok && !*abort_flag && g > 0) {
-            if (!mbar_wait(bar(kBarPFull), (g - 1) & 1)) ok = false;
-            else if (prev_first && prev_seg > 0 && !mbar_wait(bar(kBarOFree), (prev_seg - 1) & 1)) ok = false;
-            else {
-                tc_fence_after();
-                if (lane == 0) issue_O(g - 1, prev_first, prev_last);
-                __syncwarp();
-            }
-        }
+        if (ok && !*abort_flag && prev_pending && !finish_prev()) ok = false;
         if (!ok) *abort_flag = 1;
     } else {
-        // ======================================================== softmax warps 2..5 (row r = head r)
-        // Software pipeline: iteration g publishes the partial scores of tile
-        // g+1 before it runs the softmax of tile g, so the exchange with the
-        // peer overlaps a whole iteration.  Each CTA writes its fp16 partial
-        // scores into its own shared memory and the peer pulls them with
-        // ld.shared::cluster; one remote arrive per warp signals "published"
-        // and one signals "read".
+        // ======================================================== softmax warps 2..5
+        // Thread (quarter, lane): head row m = 16*quarter + lane%16 of this CTA,
+        // lane half lh = lane/16: it reads the lh partial scores, handles keys
+        // 32*lh..32*lh+31 of the row, and owns latent half lh of O.
         const int quarter = warp & 3;
-        const int r = quarter * 32 + lane;
-        const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
-        const uint32_t x_local = base + kOffX;
-        const uint32_t x_peer = mapa(x_local, peer);
-        const uint32_t xready_peer0 = mapa(bar(kBarXReady0), peer);
-        const uint32_t xread_peer0 = mapa(bar(kBarXRead0), peer);
+        const int lh = lane >> 4;
+        const int m = quarter * 16 + (lane & 15);
+        const int head = hpart * kRowsCta + m;
+        const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;  // the warp's subpartition
         const float sl2 = args.scale_log2;
         bool ok = true;
-
-        // this half of Q-hat row r -> TMEM columns kTmemQ.. (144 columns)
-        auto load_q = [&](int seq) {
-            const int u = seq * q_len + qi;
-            const uint4* src = reinterpret_cast<const uint4*>(args.q_hat + ((size_t)u * kHeads + r) * kRow);
+        TileWalk w;
+        w.init(args.plan, cl);
+        float m_used = -CUDART_INF_F, l_sum = 0.f;
+        for (int g = 0; w.valid && ok && !*abort_flag; ++g, w.advance()) {
+            if (w.first()) {
+                // Q-hat row `head`, K-half lh -> TMEM (S(g-1), the last reader of the old Q-hat, has completed).
+                const int u = w.seq * q_len + qi;
+                const uint4* src = reinterpret_cast<const uint4*>(args.q_hat + ((size_t)u * kHeads + head) * kRow);
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-                uint32_t v[32];
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t v[32];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const uint4 x = __ldg(src + half * 32 + c * 8 + j);
+                    for (int j = 0; j < 8; ++j) {
+                        const uint4 x = __ldg(src + lh * 32 + c * 8 + j);
+                        v[4 * j] = x.x; v[4 * j + 1] = x.y; v[4 * j + 2] = x.z; v[4 * j + 3] = x.w;
+                    }
+                    tmem_st32(tmem + lane_addr + kTmemQ + 32 * c, v);
+                }
+                uint32_t v[16];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint4 x = __ldg(src + 64 + lh * 4 + j);
                     v[4 * j] = x.x; v[4 * j + 1] = x.y; v[4 * j + 2] = x.z; v[4 * j + 3] = x.w;
                 }
-                tmem_st32(tmem + lane_addr + kTmemQ + 32 * c, v);
+                tmem_st16(tmem + lane_addr + kTmemQ + 128, v);
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(kBarQFull));
             }
-            uint32_t v[16];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const uint4 x = __ldg(src + 64 + half * 4 + j);
-                v[4 * j] = x.x; v[4 * j + 1] = x.y; v[4 * j + 2] = x.z; v[4 * j + 3] = x.w;
-            }
-            tmem_st16(tmem + lane_addr + kTmemQ + 128, v);
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(kBarQFull));
-        };
-        // partial S(g) out of TMEM, scaled to log2 units, published as fp16 in
-        // our buffer g & 1; own copy kept (rounded the same way) in `mine`.
-        auto fetch_send = [&](int g, uint32_t (&mine)[32]) -> bool {
-            if (!mbar_wait(bar(kBarSFull), g & 1)) return false;
+            // ---- partial S(g) of this lane half
+            if (!mbar_wait(bar(kBarSFull), g & 1)) { ok = false; break; }
             tc_fence_after();
             MLA_TRACE_POINT(7, g);
-            uint32_t v[32], v2[32];
-            tmem_ld32(tmem + lane_addr + kTmemS, v);
-            tmem_ld32(tmem + lane_addr + kTmemS + 32, v2);
+            uint32_t va[32], vb[32];
+            tmem_ld32(tmem + lane_addr + kTmemS, va);
+            tmem_ld32(tmem + lane_addr + kTmemS + 32, vb);
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(kBarSFree));
+            // ---- full scores of keys 32*lh .. +31: own partial + the other half's (lane ^ 16)
+            float s[32];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                mine[j] = pack_f16(__uint_as_float(v[2 * j]) * sl2, __uint_as_float(v[2 * j + 1]) * sl2);
-                mine[16 + j] = pack_f16(__uint_as_float(v2[2 * j]) * sl2, __uint_as_float(v2[2 * j + 1]) * sl2);
+            for (int j = 0; j < 32; ++j) {
+                const float give = __uint_as_float(lh ? va[j] : vb[j]);  // the half the partner scores
+                const float mine = __uint_as_float(lh ? vb[j] : va[j]);
+                const float other = __shfl_xor_sync(0xffffffffu, give, 16);
+                s[j] = (mine + other) * sl2;
             }
-            const int b = g & 1;
-            // the peer must have finished reading what we published in this buffer two tiles ago
-            if (g >= 2 && !mbar_wait_cluster(bar(kBarXRead0 + b), ((g - 2) >> 1) & 1)) return false;
-            MLA_TRACE_POINT(8, g);
-            const uint32_t dst = x_local + b * kXBytes + r * 128;
-#pragma unroll
-            for (int c = 0; c < 8; ++c)
-                st_shared_v4(dst + ((c ^ (r & 7)) << 4), mine[4 * c], mine[4 * c + 1], mine[4 * c + 2], mine[4 * c + 3]);
-            fence_acq_rel_cluster();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_remote(xready_peer0 + 8 * b);
-            MLA_TRACE_POINT(9, g);
-            return true;
-        };
-
-        TileWalk cur, nxt;
-        cur.init(args.plan, cl);
-        nxt = cur;
-        uint32_t mine_cur[32], mine_nxt[32];
-        if (cur.valid) {
-            load_q(cur.seq);
-            ok = fetch_send(0, mine_cur);
-            nxt.advance();
-        }
-        float m_used = -CUDART_INF_F, l_sum = 0.f;
-        int g = 0;
-        for (; cur.valid && ok && !*abort_flag; ++g) {
-            if (nxt.valid) {
-                if (nxt.seg != cur.seg) load_q(nxt.seq);  // S(g) was read: Q-hat columns are free
-                if (!fetch_send(g + 1, mine_nxt)) { ok = false; break; }
-            }
-            // ---- pull the peer's partial S(g) and add it (half 0's part first)
-            const int b = g & 1;
-            if (!mbar_wait_cluster(bar(kBarXReady0 + b), (g >> 1) & 1)) { ok = false; break; }
-            MLA_TRACE_POINT(10, g);
-            float s[kNk];
-            const uint32_t src = x_peer + b * kXBytes + r * 128;
-            uint32_t xs[32];
-#pragma unroll
-            for (int c = 0; c < 8; ++c)
-                ld_cluster_v4u(src + ((c ^ (r & 7)) << 4), xs[4 * c], xs[4 * c + 1], xs[4 * c + 2], xs[4 * c + 3]);
-#pragma unroll
-            for (int q = 0; q < 32; ++q) {
-                const float2 o = unpack_f16(xs[q]);
-                const float2 m = unpack_f16(mine_cur[q]);
-                s[2 * q] = half == 0 ? m.x + o.x : o.x + m.x;
-                s[2 * q + 1] = half == 0 ? m.y + o.y : o.y + m.y;
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive_remote(xread_peer0 + 8 * b);
-            // ---- online softmax in base 2 with lazy rescaling of O
-            const int T_b = args.seqlens[cur.seq];
+            const int T_b = args.seqlens[w.seq];
             const int n_keys = T_b - q_len + 1 + qi;  // query qi attends to keys 0..n_keys-1
-            const int key0 = cur.t * kNk;
-            if (key0 + kNk > n_keys) {
+            const int key0 = w.t * kNk + 32 * lh;
+            if (key0 + 32 > n_keys) {
 #pragma unroll
-                for (int j = 0; j < kNk; ++j)
+                for (int j = 0; j < 32; ++j)
                     if (key0 + j >= n_keys) s[j] = -CUDART_INF_F;
             }
             float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
 #pragma unroll
-            for (int j = 4; j < kNk; j += 4) {
+            for (int j = 4; j < 32; j += 4) {
                 mx0 = fmaxf(mx0, s[j]); mx1 = fmaxf(mx1, s[j + 1]);
                 mx2 = fmaxf(mx2, s[j + 2]); mx3 = fmaxf(mx3, s[j + 3]);
             }
-            const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
-            const bool first = cur.first();
+            float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+            const bool first = w.first();
             const bool grow = mx > m_used + 8.0f;  // rescale only when the max grows by > 2^8
             const float mb_new = grow ? mx : m_used;
             const float mb = (mb_new == -CUDART_INF_F) ? 0.f : mb_new;
-            uint32_t pk[32];
+            uint32_t own[16];
             float rs0 = 0.f, rs1 = 0.f;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
+            for (int j = 0; j < 16; ++j) {
                 const float p0 = ex2(s[2 * j] - mb), p1 = ex2(s[2 * j + 1] - mb);
                 rs0 += p0;
                 rs1 += p1;
-                pk[j] = pack_bf16(p0, p1);
+                own[j] = pack_bf16(p0, p1);
+            }
+            float rs = rs0 + rs1;
+            rs += __shfl_xor_sync(0xffffffffu, rs, 16);
+            uint32_t pk[32];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const uint32_t oth = __shfl_xor_sync(0xffffffffu, own[j], 16);
+                pk[j] = lh ? oth : own[j];
+                pk[16 + j] = lh ? own[j] : oth;
             }
             MLA_TRACE_POINT(11, g);
             // P(g) overwrites P(g-1) and a rescale touches O: wait for O += P(g-1) C(g-1).
@@ -511,21 +455,21 @@ __global__ void __launch_bounds__(kAttThreads, 1)
                 }
                 m_used = mx;
             }
-            l_sum += rs0 + rs1;
+            l_sum += rs;
             tmem_st32(tmem + lane_addr + kTmemP, pk);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(kBarPFull));
             MLA_TRACE_POINT(13, g);
-            // ---- epilogue at the end of a piece
-            if (cur.last()) {
-                if (!mbar_wait(bar(kBarOFull), cur.seg & 1)) { ok = false; break; }
+            // ---- epilogue at the end of a piece: this thread owns O row m, latent half lh
+            if (w.last()) {
+                if (!mbar_wait(bar(kBarOFull), w.seg & 1)) { ok = false; break; }
                 tc_fence_after();
                 const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
-                const int u = cur.seq * q_len + qi;
-                if (cur.whole) {
-                    __nv_bfloat16* dst = args.o_lat + ((size_t)u * kHeads + r) * kLat + half * kHalfLat;
+                const int u = w.seq * q_len + qi;
+                if (w.whole) {
+                    __nv_bfloat16* dst = args.o_lat + ((size_t)u * kHeads + head) * kLat + lh * kHalfLat;
 #pragma unroll 1
                     for (int c0 = 0; c0 < kHalfLat; c0 += 32) {
                         uint32_t v[32];
@@ -533,17 +477,17 @@ __global__ void __launch_bounds__(kAttThreads, 1)
                         tmem_wait_ld();
 #pragma unroll
                         for (int j = 0; j < 32; j += 8) {
-                            uint4 w;
-                            w.x = pack_bf16(__uint_as_float(v[j]) * inv, __uint_as_float(v[j + 1]) * inv);
-                            w.y = pack_bf16(__uint_as_float(v[j + 2]) * inv, __uint_as_float(v[j + 3]) * inv);
-                            w.z = pack_bf16(__uint_as_float(v[j + 4]) * inv, __uint_as_float(v[j + 5]) * inv);
-                            w.w = pack_bf16(__uint_as_float(v[j + 6]) * inv, __uint_as_float(v[j + 7]) * inv);
-                            *reinterpret_cast<uint4*>(dst + c0 + j) = w;
+                            uint4 o;
+                            o.x = pack_bf16(__uint_as_float(v[j]) * inv, __uint_as_float(v[j + 1]) * inv);
+                            o.y = pack_bf16(__uint_as_float(v[j + 2]) * inv, __uint_as_float(v[j + 3]) * inv);
+                            o.z = pack_bf16(__uint_as_float(v[j + 4]) * inv, __uint_as_float(v[j + 5]) * inv);
+                            o.w = pack_bf16(__uint_as_float(v[j + 6]) * inv, __uint_as_float(v[j + 7]) * inv);
+                            *reinterpret_cast<uint4*>(dst + c0 + j) = o;
                         }
                     }
                 } else {
-                    const int slot = cl + cur.seq;
-                    float* dst = args.part_o + (((size_t)slot * q_len + qi) * kHeads + r) * kLat + half * kHalfLat;
+                    const int slot = cl + w.seq;
+                    float* dst = args.part_o + (((size_t)slot * q_len + qi) * kHeads + head) * kLat + lh * kHalfLat;
 #pragma unroll 1
                     for (int c0 = 0; c0 < kHalfLat; c0 += 32) {
                         uint32_t v[32];
@@ -551,13 +495,13 @@ __global__ void __launch_bounds__(kAttThreads, 1)
                         tmem_wait_ld();
 #pragma unroll
                         for (int j = 0; j < 32; j += 4) {
-                            float4 w = make_float4(__uint_as_float(v[j]) * inv, __uint_as_float(v[j + 1]) * inv,
+                            float4 o = make_float4(__uint_as_float(v[j]) * inv, __uint_as_float(v[j + 1]) * inv,
                                                    __uint_as_float(v[j + 2]) * inv, __uint_as_float(v[j + 3]) * inv);
-                            *reinterpret_cast<float4*>(dst + c0 + j) = w;
+                            *reinterpret_cast<float4*>(dst + c0 + j) = o;
                         }
                     }
-                    if (half == 0)
-                        args.part_lse[((size_t)slot * q_len + qi) * kHeads + r] =
+                    if (lh == 0)
+                        args.part_lse[((size_t)slot * q_len + qi) * kHeads + head] =
                             l_sum > 0.f ? m_used + __log2f(l_sum) : -CUDART_INF_F;
                 }
                 tc_fence_before();
@@ -566,11 +510,6 @@ __global__ void __launch_bounds__(kAttThreads, 1)
                 m_used = -CUDART_INF_F;
                 l_sum = 0.f;
             }
-            // advance the pipeline
-#pragma unroll
-            for (int j = 0; j < 32; ++j) mine_cur[j] = mine_nxt[j];
-            cur = nxt;
-            if (nxt.valid) nxt.advance();
         }
         if (!ok) *abort_flag = 1;
     }
@@ -579,8 +518,6 @@ __global__ void __launch_bounds__(kAttThreads, 1)
     tc_fence_before();
     __syncthreads();
     if (warp == 1) tmem_dealloc(tmem, kTmemCols);
-    // The peer may still read our barriers / write our X buffers until it is done.
-    cluster_sync();
 }
 
 // ------------------------------------------------------------------ plan
