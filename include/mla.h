@@ -106,7 +106,7 @@ size_t mla_workspace_bytes(const mla_dims_t* dims, int32_t B, int32_t q_len);
 
 /* ---------------------------------------------------------------- decode
  * One absorbed-MLA decode step for B sequences with q_len query tokens each
- * (q_len = 1 plain decode; 2..4 speculative verify, causal among the new
+ * (q_len = 1 plain decode; 2..16 speculative verify, causal among the new
  * tokens).  seqlens[b] counts cached tokens INCLUDING the q_len new ones,
  * which must already be appended; query i sits at position
  * m = seqlens[b] - q_len + i and attends to keys 0..m.
@@ -128,17 +128,21 @@ int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_rope,
  *         CUDA kernels otherwise), 1 = force the tensor-core path
  *         (MLA_ERR_UNSUPPORTED if it cannot run), 2 = force the generic path.
  *   num_pairs: CTA pairs (clusters) of the attention grid (0 = one per two SMs).
- *   overhead_tiles: scheduling cost charged per sequence, in 64-key tiles
+ *   overhead_tiles: scheduling cost charged per query token (each of the
+ *         B * q_len tokens is scheduled on its own), in 64-key tiles
  *         (negative = default).
+ *   min_tiles: smallest piece of a token's keys one cluster takes, in 64-key tiles
+ *         (0 = default); larger values mean fewer split partials to merge.
  *   events / n_events: optional caller-created cudaEvent_t handles; when
  *         n_events >= MLA_NUM_EVENTS, mla_decode_ex records them on `stream`
  *         at the stage boundaries listed below, so a caller can time each
  *         kernel with cudaEventElapsedTime.  The library does not own them.
- *   All-zero options (path 0, num_pairs 0, overhead_tiles 0, no events) are valid. */
+ *   All-zero options are valid (overhead_tiles 0 charges nothing per sequence). */
 typedef struct {
     int32_t path;
     int32_t num_pairs;
     int32_t overhead_tiles;
+    int32_t min_tiles;
     int32_t n_events;
     void* const* events;
 } mla_decode_opts_t;
@@ -174,8 +178,8 @@ int mla_decode_ex(const mla_dims_t* dims, const void* q_nope, const void* q_rope
  * image, which every GPU that loads the library keeps until the process
  * exits.  A batch whose mla_workspace_bytes() exceeds 64 MiB is rejected with
  * MLA_ERR_WORKSPACE before anything is launched; on a 148-SM B200 the limit
- * is 88 sequences at q_len = 1, 26 at q_len = 2, 5 at q_len = 3 (q_len = 4
- * does not fit).  The call allocates nothing
+ * is B * q_len <= 88 query tokens (88 sequences at q_len = 1, 44 at
+ * q_len = 2, 22 at q_len = 4).  The call allocates nothing
  * and calls no allocating routine.
  *
  * The first call on each device looks up the array's device address

@@ -45,7 +45,8 @@ class Cache(ctypes.Structure):
 
 class Opts(ctypes.Structure):
     _fields_ = [("path", ctypes.c_int32), ("num_pairs", ctypes.c_int32), ("overhead_tiles", ctypes.c_int32),
-                ("n_events", ctypes.c_int32), ("events", ctypes.POINTER(ctypes.c_void_p))]
+                ("min_tiles", ctypes.c_int32), ("n_events", ctypes.c_int32),
+                ("events", ctypes.POINTER(ctypes.c_void_p))]
 
 
 class MLAError(RuntimeError):
@@ -133,9 +134,9 @@ class Library:
         return Cache(cache.data_ptr(), cache.shape[0], cache.shape[1], cache.stride(0), cache.stride(1))
 
     @staticmethod
-    def opts(path=PATH_AUTO, num_pairs=0, overhead_tiles=-1, events=None) -> Opts:
+    def opts(path=PATH_AUTO, num_pairs=0, overhead_tiles=-1, min_tiles=0, events=None) -> Opts:
         """``events``: MLA_NUM_EVENTS recorded torch.cuda.Event objects (stage timing)."""
-        o = Opts(path, num_pairs, overhead_tiles, 0, None)
+        o = Opts(path, num_pairs, overhead_tiles, min_tiles, 0, None)
         if events is not None:
             arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
             o.events = ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p))

@@ -52,6 +52,7 @@ int check_dims(const mla_dims_t* d, Problem* p) {
         return fail(MLA_ERR_SHAPE, "head dimensions must be positive (H=%d d_c=%d d_r=%d d_n=%d d_v=%d)", d->H,
                     d->d_c, d->d_r, d->d_n, d->d_v);
     if (d->d_r % 2) return fail(MLA_ERR_SHAPE, "d_r must be even (RoPE pairs), got %d", d->d_r);
+    if (d->d_r > 128) return fail(MLA_ERR_SHAPE, "d_r > 128 is not supported");
     if (d->d_c > 1024) return fail(MLA_ERR_SHAPE, "d_c > 1024 is not supported");
     if (d->dtype != MLA_DTYPE_BF16 && d->dtype != MLA_DTYPE_F32) return fail(MLA_ERR_ARG, "unknown dtype %d", d->dtype);
     if (!(d->rope_base > 0.f)) return fail(MLA_ERR_ARG, "rope_base must be > 0");
@@ -66,6 +67,8 @@ int check_dims(const mla_dims_t* d, Problem* p) {
     p->scale = d->softmax_scale > 0.f ? d->softmax_scale : 1.0f / sqrtf((float)(d->d_n + d->d_r));
     p->B = 0;
     p->q_len = 1;
+    for (int k = 0; k < 64; ++k)
+        p->rope.inv_freq[k] = (k < d->d_r / 2) ? pow((double)d->rope_base, -2.0 * k / (double)d->d_r) : 0.0;
     return MLA_OK;
 }
 
@@ -105,7 +108,8 @@ int choose_path(const Problem& p, int q_len, const mla_decode_opts_t* o, bool* f
 }
 
 int pairs_for(const mla_decode_opts_t* o) {
-    const int n = (o && o->num_pairs > 0) ? o->num_pairs : sm100_default_pairs();
+    int n = (o && o->num_pairs > 0) ? o->num_pairs : sm100_default_pairs();
+    if (n > 1024) n = 1024;  // the split combine handles at most 1024 pieces per sequence
     return n > 0 ? n : 1;
 }
 
@@ -259,7 +263,7 @@ int mla_attend_latent(const mla_dims_t* dims, const void* q_hat, const mla_cache
             return fail(MLA_ERR_WORKSPACE, "attend workspace needs %zu bytes (16-byte aligned), got %zu", need,
                         workspace_bytes);
         e = sm100_attend(p, q_hat, cv, seqlens, o_lat, workspace, workspace_bytes, pairs,
-                         opts ? opts->overhead_tiles : -1, status, (cudaStream_t)stream);
+                         opts ? opts->overhead_tiles : -1, opts ? opts->min_tiles : 0, status, (cudaStream_t)stream);
     } else {
         e = generic_attend(p, q_hat, cv, seqlens, o_lat, status, (cudaStream_t)stream);
     }
@@ -326,11 +330,19 @@ int mla_decode_ex(const mla_dims_t* dims, const void* q_nope, const void* q_rope
     cudaError_t e;
     ev.record(MLA_EV_START, st);
     if (fast) {
-        e = sm100_absorb(p, q_nope, q_rope, W_UK, seqlens, q_hat, st);
+        PlanRequest pr;
+        pr.plan = ws + L.attend;
+        pr.o_lat = o_lat;
+        pr.T_max = cv.T_max;
+        pr.clusters = pairs;
+        pr.overhead_tiles = opts ? opts->overhead_tiles : -1;
+        pr.min_tiles = opts ? opts->min_tiles : 0;
+        e = sm100_absorb(p, q_nope, q_rope, W_UK, seqlens, q_hat, st, &pr);
         ev.record(MLA_EV_ABSORB_DONE, st);
         if (e == cudaSuccess)
             e = sm100_attend(p, q_hat, cv, seqlens, o_lat, ws + L.attend, L.total - L.attend, pairs,
-                             opts ? opts->overhead_tiles : -1, status, st, &ev);
+                             opts ? opts->overhead_tiles : -1, opts ? opts->min_tiles : 0, status, st, &ev,
+                             /*plan_ready=*/true);
         ev.record(MLA_EV_COMBINE_DONE, st);
         if (e == cudaSuccess) e = sm100_project(p, o_lat, W_UV, B * q_len, out, st);
     } else {

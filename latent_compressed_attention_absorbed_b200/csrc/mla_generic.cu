@@ -39,7 +39,7 @@ __global__ void append_kernel(Problem p, const T* __restrict__ c_kv, const T* __
     for (int e = threadIdx.x; e < p.d_c; e += blockDim.x) row[e] = c[e];
     for (int kk = threadIdx.x; kk < p.d_r / 2; kk += blockDim.x) {
         float y0, y1;
-        mla_rope_pair(ld(k, 2 * kk), ld(k, 2 * kk + 1), kk, p.d_r, t, p.rope_base, &y0, &y1);
+        mla_rope_rotate(ld(k, 2 * kk), ld(k, 2 * kk + 1), p.rope.inv_freq[kk], t, &y0, &y1);
         st(row, p.d_c + 2 * kk, y0);
         st(row, p.d_c + 2 * kk + 1, y1);
     }
@@ -67,7 +67,7 @@ __global__ void absorb_kernel(Problem p, const T* __restrict__ q_nope, const T* 
     const T* qr = q_rope + ((size_t)u * p.H + h) * p.d_r;
     for (int kk = threadIdx.x; kk < p.d_r / 2; kk += blockDim.x) {
         float y0, y1;
-        mla_rope_pair(ld(qr, 2 * kk), ld(qr, 2 * kk + 1), kk, p.d_r, m, p.rope_base, &y0, &y1);
+        mla_rope_rotate(ld(qr, 2 * kk), ld(qr, 2 * kk + 1), p.rope.inv_freq[kk], m, &y0, &y1);
         st(out, p.d_c + 2 * kk, y0);
         st(out, p.d_c + 2 * kk + 1, y1);
     }

@@ -7,6 +7,7 @@
 #include <stdint.h>
 
 #include "mla.h"
+#include "mla_rope.cuh"
 
 namespace mla {
 
@@ -17,6 +18,7 @@ struct Problem {
     float rope_base;
     float scale;  // softmax scale (already resolved)
     int B, q_len;
+    RopeTable rope;  // inverse RoPE frequencies (fp64, host-computed)
 };
 
 // Optional stage-boundary events of one decode call (see MLA_EV_* in mla.h).
@@ -72,11 +74,18 @@ size_t generic_workspace_bytes(const Problem& p);
 bool sm100_supported(const Problem& p, int q_len);
 cudaError_t sm100_append(const Problem& p, const void* c_kv, const void* k_rope, const int32_t* pos,
                          int n_tok, const CacheView& cache, int* status, cudaStream_t st);
+// When given, the absorb GEMM also writes the attention's split plan.
+struct PlanRequest {
+    void* plan;   // start of the attention workspace
+    void* o_lat;  // zeroed for sequences with an invalid length
+    int T_max, clusters, overhead_tiles, min_tiles;
+};
 cudaError_t sm100_absorb(const Problem& p, const void* q_nope, const void* q_rope, const void* W_UK,
-                         const int32_t* seqlens, void* q_hat, cudaStream_t st);
+                         const int32_t* seqlens, void* q_hat, cudaStream_t st, const PlanRequest* plan = nullptr);
 cudaError_t sm100_attend(const Problem& p, const void* q_hat, const CacheView& cache, const int32_t* seqlens,
                          void* o_lat, void* workspace, size_t ws_bytes, int num_pairs, int overhead_tiles,
-                         int* status, cudaStream_t st, const Events* events = nullptr);
+                         int min_tiles, int* status, cudaStream_t st, const Events* events = nullptr,
+                         bool plan_ready = false);
 cudaError_t sm100_project(const Problem& p, const void* o_lat, const void* W_UV, int rows, void* out,
                           cudaStream_t st);
 size_t sm100_attend_workspace_bytes(const Problem& p, int num_pairs);

@@ -20,10 +20,10 @@
 
 namespace {
 
-// 64 MiB.  On a 148-SM B200 this holds the decode workspace of up to 88
-// sequences at q_len = 1, 26 at q_len = 2 and 5 at q_len = 3 (the split-KV
-// partials take (SMs/2 + B) * q_len * 256 KiB); q_len = 4 does not fit.
-// Larger batches are rejected before anything is launched.
+// 64 MiB.  On a 148-SM B200 this holds the decode workspace of up to
+// B * q_len = 88 query tokens: each token takes about 529 KiB (Q-hat, o_lat
+// and one split-KV partial slot) on top of 74 fixed partial slots of
+// 256.5 KiB.  Larger batches are rejected before anything is launched.
 constexpr size_t kScratchBytes = size_t(64) << 20;
 
 static __device__ __align__(256) unsigned char g_decode_scratch[kScratchBytes];

@@ -6,6 +6,8 @@
 #include <math.h>
 #include <string.h>
 
+#include <utility>
+
 #include "mla_internal.h"
 #include "mla_rope.cuh"
 #include "sm100_attend.cuh"
@@ -62,7 +64,7 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64
 // One warp per new token: 16-byte copies of the 512 latent values and the
 // RoPE rotation of the 64-wide key at its position (one pair per lane).
 __global__ void append_v3_kernel(const __nv_bfloat16* __restrict__ c_kv, const __nv_bfloat16* __restrict__ k_rope,
-                                 const int32_t* __restrict__ pos, int B, int n_tok, CacheView cache, float base,
+                                 const int32_t* __restrict__ pos, int B, int n_tok, CacheView cache, RopeTable rope,
                                  int* status) {
     const int gw = (blockIdx.x * blockDim.x + threadIdx.x) / 32;
     const int lane = threadIdx.x & 31;
@@ -81,7 +83,7 @@ __global__ void append_v3_kernel(const __nv_bfloat16* __restrict__ c_kv, const _
     dst[lane + 32] = src[lane + 32];
     const __nv_bfloat162 k2 = reinterpret_cast<const __nv_bfloat162*>(k_rope + (size_t)gw * kRope)[lane];
     float y0, y1;
-    mla_rope_pair(__low2float(k2), __high2float(k2), lane, kRope, t, base, &y0, &y1);
+    mla_rope_rotate(__low2float(k2), __high2float(k2), rope.inv_freq[lane], t, &y0, &y1);
     reinterpret_cast<__nv_bfloat162*>(row + kLat)[lane] = __floats2bfloat162_rn(y0, y1);
 }
 
@@ -101,7 +103,42 @@ cudaError_t set_smem(K kernel, int bytes, bool (&done)[kMaxDev]) {
 }
 bool g_smem_absorb[kMaxDev], g_smem_project[kMaxDev], g_smem_attend[kMaxDev];
 
+// Launch with programmatic dependent launch allowed: the kernel may start
+// while the previous kernel on the stream is finishing; it calls
+// griddepcontrol.wait before touching anything that kernel may write.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, int cluster_x,
+                       Args&&... args) {
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    int n = 0;
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+    if (cluster_x > 1) {
+        attr[n].id = cudaLaunchAttributeClusterDimension;
+        attr[n].val.clusterDim.x = cluster_x;
+        attr[n].val.clusterDim.y = 1;
+        attr[n].val.clusterDim.z = 1;
+        ++n;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = n;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 constexpr int kAbsorbStages = 2;
+// Rows of the A tile a GEMM CTA loads: all 128 when the batch fills them,
+// else the batch rounded up to 16 (the MMA still computes 128 rows; the rows
+// past the batch are never stored).
+int plan_ovh(int overhead_tiles) { return overhead_tiles < 0 ? 2 : overhead_tiles; }
+int plan_min_units(int min_tiles) { return min_tiles > 0 ? min_tiles : 1; }
+int gemm_a_rows(int rows) { return rows >= 128 ? 128 : ((rows + 15) / 16) * 16; }
 constexpr int kProjStages = 4;
 constexpr int kProjNT = 64;
 
@@ -111,7 +148,7 @@ bool sm100_supported(const Problem& p, int q_len) {
     if (p.dtype != MLA_DTYPE_BF16 || p.H != kHeads || p.d_c != kLat || p.d_r != kRope || p.d_n != 128 ||
         p.d_v != 128)
         return false;
-    if (q_len < 1 || q_len > 4) return false;
+    if (q_len < 1 || q_len > 16) return false;
     int dev = 0, major = 0, minor = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return false;
     cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
@@ -127,16 +164,16 @@ cudaError_t sm100_append(const Problem& p, const void* c_kv, const void* k_rope,
     const int threads = 128;
     const int blocks = (warps * 32 + threads - 1) / threads;
     append_v3_kernel<<<blocks, threads, 0, st>>>((const __nv_bfloat16*)c_kv, (const __nv_bfloat16*)k_rope, pos, p.B,
-                                                 n_tok, cache, p.rope_base, status);
+                                                 n_tok, cache, p.rope, status);
     return cudaGetLastError();
 }
 
 cudaError_t sm100_absorb(const Problem& p, const void* q_nope, const void* q_rope, const void* W_UK,
-                         const int32_t* seqlens, void* q_hat, cudaStream_t st) {
+                         const int32_t* seqlens, void* q_hat, cudaStream_t st, const PlanRequest* plan) {
     const int rows = p.B * p.q_len;
     CUtensorMap mA, mB;
     // A: q_nope viewed as [rows][H][128]; box 64 x 1 x 128 rows.
-    if (!make_map(&mA, q_nope, 128, kHeads, rows, 128 * 2, (uint64_t)kHeads * 128 * 2, 64, 1, 128,
+    if (!make_map(&mA, q_nope, 128, kHeads, rows, 128 * 2, (uint64_t)kHeads * 128 * 2, 64, 1, gemm_a_rows(rows),
                   CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
     // B: W_UK viewed as [H][128 (d)][512 (c)]; box 64 c x 64 d x 1.
@@ -156,18 +193,28 @@ cudaError_t sm100_absorb(const Problem& p, const void* q_nope, const void* q_rop
     a.q_rope = (const __nv_bfloat16*)q_rope;
     a.seqlens = seqlens;
     a.q_len = p.q_len;
-    a.rope_base = p.rope_base;
+    a.rope = p.rope;
     a.status = device_status_ptr();
+    a.a_rows = gemm_a_rows(rows);
+    a.plan = nullptr;
+    if (plan) {
+        a.plan = static_cast<Plan*>(plan->plan);
+        a.plan_B = p.B;
+        a.plan_T_max = plan->T_max;
+        a.plan_clusters = plan->clusters;
+        a.plan_ovh = plan_ovh(plan->overhead_tiles);
+        a.plan_min_units = plan_min_units(plan->min_tiles);
+        a.plan_olat = static_cast<__nv_bfloat16*>(plan->o_lat);
+    }
     dim3 grid(kHeads, kLat / 256, (rows + 127) / 128);
-    kern<<<grid, 128, Cfg::kSmem, st>>>(mA, mB, a);
-    return cudaGetLastError();
+    return launch_pdl(kern, grid, dim3(128), Cfg::kSmem, st, 1, mA, mB, a);
 }
 
 cudaError_t sm100_project(const Problem& p, const void* o_lat, const void* W_UV, int rows, void* out,
                           cudaStream_t st) {
     CUtensorMap mA, mB;
     // A: o_lat viewed as [rows][H][512]; box 64 x 1 x 128.
-    if (!make_map(&mA, o_lat, kLat, kHeads, rows, kLat * 2, (uint64_t)kHeads * kLat * 2, 64, 1, 128,
+    if (!make_map(&mA, o_lat, kLat, kHeads, rows, kLat * 2, (uint64_t)kHeads * kLat * 2, 64, 1, gemm_a_rows(rows),
                   CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
     // B: W_UV viewed as [H][128 (d)][512 (c)]; box 64 c x NT d x 1 (K-major).
@@ -180,6 +227,7 @@ cudaError_t sm100_project(const Problem& p, const void* o_lat, const void* W_UV,
     if (e != cudaSuccess) return e;
     GemmArgs a;
     memset(&a, 0, sizeof(a));
+    a.plan = nullptr;
     a.rows = rows;
     a.H = kHeads;
     a.ld_out = 128;
@@ -187,22 +235,25 @@ cudaError_t sm100_project(const Problem& p, const void* o_lat, const void* W_UV,
     a.out = (__nv_bfloat16*)out;
     a.status = device_status_ptr();
     a.q_len = 1;
+    a.a_rows = gemm_a_rows(rows);
     dim3 grid(kHeads, 128 / kProjNT, (rows + 127) / 128);
-    kern<<<grid, 128, Cfg::kSmem, st>>>(mA, mB, a);
-    return cudaGetLastError();
+    return launch_pdl(kern, grid, dim3(128), Cfg::kSmem, st, 1, mA, mB, a);
 }
 
 // Workspace of the attention step: plan, fp32 partials and LSEs.
 static size_t attend_layout(const Problem& p, int clusters, size_t* off_part, size_t* off_lse) {
     Carve c(nullptr);
-    c.take(sizeof(Plan) + sizeof(int) * (p.B + 1));
-    const size_t slots = (size_t)clusters + p.B;
+    const size_t units = (size_t)p.B * p.q_len;  // one per query token
+    c.take(sizeof(Plan) + sizeof(int) * (2 * units + 1));
+    const size_t slots = (size_t)clusters + units;
     *off_part = c.off;
-    c.take(slots * p.q_len * kHeads * kLat * sizeof(float));
+    c.take(slots * kHeads * kLat * sizeof(float));
     *off_lse = c.off;
-    c.take(slots * p.q_len * kHeads * sizeof(float));
+    c.take(slots * kHeads * sizeof(float));
     return c.off;
 }
+
+void* sm100_plan_ptr(void* attend_workspace) { return attend_workspace; }
 
 size_t sm100_attend_workspace_bytes(const Problem& p, int num_pairs) {
     size_t a, b;
@@ -211,7 +262,7 @@ size_t sm100_attend_workspace_bytes(const Problem& p, int num_pairs) {
 
 cudaError_t sm100_attend(const Problem& p, const void* q_hat, const CacheView& cache, const int32_t* seqlens,
                          void* o_lat, void* workspace, size_t ws_bytes, int num_pairs, int overhead_tiles,
-                         int* status, cudaStream_t st, const Events* events) {
+                         int min_tiles, int* status, cudaStream_t st, const Events* events, bool plan_ready) {
     const int clusters = num_pairs;
     size_t off_part, off_lse;
     const size_t need = attend_layout(p, clusters, &off_part, &off_lse);
@@ -223,10 +274,13 @@ cudaError_t sm100_attend(const Problem& p, const void* q_hat, const CacheView& c
     if (!make_map(&mC, cache.data, kRow, cache.T_max, p.B, stt, sb, 64, kNk, 1, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
 
-    const int ovh = overhead_tiles < 0 ? 2 : overhead_tiles;
-    mla_plan_kernel<<<1, 1024, 0, st>>>(seqlens, p.B, p.q_len, cache.T_max, clusters, ovh, 1, plan, status);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
+    cudaError_t e;
+    if (!plan_ready) {
+        mla_plan_kernel<<<1, 32, 0, st>>>(seqlens, p.B, p.q_len, cache.T_max, clusters, plan_ovh(overhead_tiles),
+                                          plan_min_units(min_tiles), plan, status, (__nv_bfloat16*)o_lat);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
 
     e = set_smem(mla_attend_kernel, kAttSmem, g_smem_attend);
     if (e != cudaSuccess) return e;
@@ -242,28 +296,26 @@ cudaError_t sm100_attend(const Problem& p, const void* q_hat, const CacheView& c
     a.part_lse = reinterpret_cast<float*>(ws + off_lse);
     a.status = status;
 
-    cudaLaunchConfig_t cfg;
-    memset(&cfg, 0, sizeof(cfg));
-    const int csize = 2 * p.q_len;
-    cfg.gridDim = dim3(clusters * csize, 1, 1);
-    cfg.blockDim = dim3(kAttThreads, 1, 1);
-    cfg.dynamicSmemBytes = kAttSmem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = csize;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
     if (events) events->record(MLA_EV_ATTEND_BEGIN, st);
-    e = cudaLaunchKernelEx(&cfg, mla_attend_kernel, mC, a);
+    e = launch_pdl(mla_attend_kernel, dim3(clusters * 2), dim3(kAttThreads), kAttSmem, st, 2, mC, a);
     if (e != cudaSuccess) return e;
     if (events) events->record(MLA_EV_ATTEND_END, st);
 
-    const int warps = p.B * p.q_len * kHeads;
-    mla_combine_kernel<<<(warps * 32 + 255) / 256, 256, 0, st>>>(plan, a.part_o, a.part_lse, p.q_len,
-                                                                 (__nv_bfloat16*)o_lat);
+    // Split units number at most min(B * q_len, clusters - 1).  With many
+    // pieces per unit (small batches) the warp-per-piece merge is used.
+    const int units = p.B * p.q_len;
+    const int max_split = units < clusters ? units : clusters;
+    const Plan* cplan = plan;
+    const float* po = a.part_o;
+    const float* pl = a.part_lse;
+    __nv_bfloat16* ol = (__nv_bfloat16*)o_lat;
+    if (4 * units < clusters)
+        e = launch_pdl(mla_combine_kernel<8, 1>, dim3(max_split * (kLat / 4)), dim3(1024), 0, st, 1, cplan, po, pl,
+                       ol);
+    else
+        e = launch_pdl(mla_combine_kernel<1, 2>, dim3(max_split * (kLat / 8)), dim3(256), 0, st, 1, cplan, po, pl,
+                       ol);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

@@ -18,6 +18,7 @@
 #include <cuda_bf16.h>
 
 #include "mla_rope.cuh"
+#include "sm100_attend.cuh"
 #include "sm100_ptx.cuh"
 
 namespace mla {
@@ -33,8 +34,13 @@ struct GemmArgs {
     const __nv_bfloat16* q_rope;  // [rows][H][64]
     const int32_t* seqlens;       // [B]
     int q_len;
-    float rope_base;
+    RopeTable rope;
+    int a_rows;       // rows of each A box (multiple of 16, <= 128)
     int* status;
+    // split plan of the attention step, written by warp 2 of CTA (0,0,0) when non-null
+    Plan* plan;
+    int plan_B, plan_T_max, plan_clusters, plan_ovh, plan_min_units;
+    __nv_bfloat16* plan_olat;
 };
 
 template <int KCH, int NT, bool B_MN, int STAGES, bool ROPE>
@@ -90,16 +96,12 @@ __global__ void __launch_bounds__(128, 1)
 
     if (warp == 0 && lane == 0) {
         // ---------------- producer
-        for (int kc = 0; kc < KCH; ++kc) {
-            const int s = kc % STAGES;
-            if (kc >= STAGES && !mbar_wait(empty_bar(s), ((kc / STAGES) - 1) & 1)) {
-                *abort_flag = 1;
-                break;
-            }
-            const uint32_t a_dst = base + s * C::kStage;
-            const uint32_t b_dst = a_dst + C::kABytes;
-            mbar_arrive_expect_tx(full_bar(s), C::kStage);
-            tma_load_3d(a_dst, &mapA, full_bar(s), kc * 64, h, m0);
+        // The weight tiles (B) of the first stages are requested before the
+        // grid dependency wait: weights are never written by the kernel
+        // that precedes this one.  The activations (A) only after it.
+        constexpr int kPre = KCH < STAGES ? KCH : STAGES;
+        auto load_B = [&](int kc, int s) {
+            const uint32_t b_dst = base + s * C::kStage + C::kABytes;
             if (B_MN) {
 #pragma unroll
                 for (int j = 0; j < NT / 64; ++j)
@@ -107,6 +109,24 @@ __global__ void __launch_bounds__(128, 1)
             } else {
                 tma_load_3d(b_dst, &mapB, full_bar(s), kc * 64, n0, h);
             }
+        };
+        for (int kc = 0; kc < kPre; ++kc) {
+            mbar_arrive_expect_tx(full_bar(kc), args.a_rows * 128 + C::kBBytes);
+            load_B(kc, kc);
+        }
+        pdl_wait();
+        pdl_trigger();
+        for (int kc = 0; kc < KCH; ++kc) {
+            const int s = kc % STAGES;
+            if (kc >= kPre) {
+                if (!mbar_wait(empty_bar(s), ((kc / STAGES) - 1) & 1)) {
+                    *abort_flag = 1;
+                    break;
+                }
+                mbar_arrive_expect_tx(full_bar(s), args.a_rows * 128 + C::kBBytes);
+                load_B(kc, s);
+            }
+            tma_load_3d(base + s * C::kStage, &mapA, full_bar(s), kc * 64, h, m0);
         }
     } else if (warp == 1 && lane == 0) {
         // ---------------- MMA issuer
@@ -130,6 +150,11 @@ __global__ void __launch_bounds__(128, 1)
         }
         mma_commit(done_bar);
     }
+    // Nothing is written before the kernels this one depends on have completed.
+    pdl_wait();
+    if (warp == 2 && args.plan && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0)
+        mla_plan_warp(args.seqlens, args.plan_B, args.q_len, args.plan_T_max, args.plan_clusters, args.plan_ovh,
+                      args.plan_min_units, args.plan, args.status, args.plan_olat, lane);
     __syncwarp();
 
     // ---------------- epilogue: all four warps, TMEM lane quarter = warp
@@ -158,28 +183,19 @@ __global__ void __launch_bounds__(128, 1)
     } else if (threadIdx.x == 0) {
         atomicOr(args.status, MLA_STATUS_TIMEOUT);
     }
-    if (ROPE && blockIdx.y == 0 && row < args.rows) {
-        // q_hat[u][h][512 + :] = RoPE(q_rope[u][h], m_u), m_u = seqlens[b] - q_len + i
-        const int b = row / args.q_len, i = row % args.q_len;
-        const int m = args.seqlens[b] - args.q_len + i;
-        const __nv_bfloat16* src = args.q_rope + ((size_t)row * args.H + h) * 64;
-        __nv_bfloat16* dst = args.out + ((size_t)row * args.H + h) * args.ld_out + 512;
-#pragma unroll 1
-        for (int k = 0; k < 32; k += 4) {
-            uint4 o;
-            uint32_t w[4];
-            for (int t = 0; t < 4; ++t) {
-                const float x0 = __bfloat162float(src[2 * (k + t)]);
-                const float x1 = __bfloat162float(src[2 * (k + t) + 1]);
-                float y0, y1;
-                mla_rope_pair(x0, x1, k + t, 64, m, args.rope_base, &y0, &y1);
-                w[t] = pack_bf16(y0, y1);
-            }
-            o.x = w[0];
-            o.y = w[1];
-            o.z = w[2];
-            o.w = w[3];
-            *reinterpret_cast<uint4*>(dst + 2 * k) = o;
+    if (ROPE) {
+        // q_hat[u][h][512 + 2k..] = RoPE(q_rope[u][h], m_u) for the rows of this tile, one pair per item,
+        // pairs 16y..16y+15 in the CTA with N-tile y: m_u = seqlens[b] - q_len + i.
+        const int nrows = min(128, args.rows - m0);
+        for (int item = threadIdx.x; item < nrows * 16; item += blockDim.x) {
+            const int u = m0 + item / 16, k = 16 * blockIdx.y + item % 16;
+            const int b = u / args.q_len, i = u % args.q_len;
+            const int m = args.seqlens[b] - args.q_len + i;
+            const __nv_bfloat162 x = reinterpret_cast<const __nv_bfloat162*>(args.q_rope + ((size_t)u * args.H + h) * 64)[k];
+            float y0, y1;
+            mla_rope_rotate(__low2float(x), __high2float(x), args.rope.inv_freq[k], m, &y0, &y1);
+            reinterpret_cast<__nv_bfloat162*>(args.out + ((size_t)u * args.H + h) * args.ld_out + 512)[k] =
+                __floats2bfloat162_rn(y0, y1);
         }
     }
     tc_fence_before();

@@ -85,6 +85,10 @@ SMALL_CASES = [
     ((513, 2000, 5), 3, 7),
     ((257, 1024), 4, 5),
     ((4096,), 1, 64),          # long sequence cut in many pieces
+    ((4000,) + (5,) * 24, 1, 0),  # one long sequence among short ones: many pieces in a large batch
+    ((3000, 2, 900) * 3, 2, 0),   # ragged verify batch
+    ((1500, 9, 260), 8, 0),       # long verify window: 8 query tokens per sequence
+    ((16, 700), 16, 5),           # the largest q_len; the first sequence holds only its new tokens
 ]
 
 
