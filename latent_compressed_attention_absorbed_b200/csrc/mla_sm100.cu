@@ -19,6 +19,11 @@
 extern "C" int mla_trace_read(void* host, size_t bytes) {
     return cudaMemcpyFromSymbol(host, mla::sm100::g_mla_trace, bytes) == cudaSuccess ? 0 : -4;
 }
+extern "C" int mla_trace_clear(void) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, mla::sm100::g_mla_trace) != cudaSuccess) return -4;
+    return cudaMemset(p, 0, sizeof(mla::sm100::g_mla_trace)) == cudaSuccess ? 0 : -4;
+}
 #endif
 
 namespace mla {
@@ -240,8 +245,13 @@ cudaError_t sm100_project(const Problem& p, const void* o_lat, const void* W_UV,
     return launch_pdl(kern, grid, dim3(128), Cfg::kSmem, st, 1, mA, mB, a);
 }
 
+// Clusters of the attention grid: at least one per query token (a group of
+// q_len clusters streams one sequence piece, one cluster per token).
+static int attend_clusters(int pairs, int q_len) { return pairs < q_len ? q_len : pairs; }
+
 // Workspace of the attention step: plan, fp32 partials and LSEs.
-static size_t attend_layout(const Problem& p, int clusters, size_t* off_part, size_t* off_lse) {
+static size_t attend_layout(const Problem& p, int pairs, size_t* off_part, size_t* off_lse) {
+    const int clusters = attend_clusters(pairs, p.q_len);
     Carve c(nullptr);
     const size_t units = (size_t)p.B * p.q_len;  // one per query token
     c.take(sizeof(Plan) + sizeof(int) * (2 * units + 1));
@@ -263,15 +273,22 @@ size_t sm100_attend_workspace_bytes(const Problem& p, int num_pairs) {
 cudaError_t sm100_attend(const Problem& p, const void* q_hat, const CacheView& cache, const int32_t* seqlens,
                          void* o_lat, void* workspace, size_t ws_bytes, int num_pairs, int overhead_tiles,
                          int min_tiles, int* status, cudaStream_t st, const Events* events, bool plan_ready) {
-    const int clusters = num_pairs;
+    const int clusters = attend_clusters(num_pairs, p.q_len);
     size_t off_part, off_lse;
     const size_t need = attend_layout(p, clusters, &off_part, &off_lse);
     if (ws_bytes < need) return cudaErrorInvalidValue;
     char* ws = static_cast<char*>(workspace);
     Plan* plan = reinterpret_cast<Plan*>(ws);
-    CUtensorMap mC;
+    // Cache as [B][T_max][576]: latent boxes of 64 columns (SW128), RoPE half
+    // boxes of 32 columns (SW64), 64 keys each, and 256-column boxes for the
+    // L2 prefetch.
+    CUtensorMap mLat, mRope, mPf, mQR;
     const uint64_t sb = (uint64_t)cache.stride_b * 2, stt = (uint64_t)cache.stride_t * 2;
-    if (!make_map(&mC, cache.data, kRow, cache.T_max, p.B, stt, sb, 64, kNk, 1, CU_TENSOR_MAP_SWIZZLE_128B))
+    if (!make_map(&mLat, cache.data, kRow, cache.T_max, p.B, stt, sb, 64, kNk, 1, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&mRope, cache.data, kRow, cache.T_max, p.B, stt, sb, kHalfRope, kNk, 1, CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !make_map(&mPf, cache.data, kRow, cache.T_max, p.B, stt, sb, kHalfLat, kNk, 1, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_map(&mQR, q_hat, kRow, kHeads, (uint64_t)p.B * p.q_len, kRow * 2, (uint64_t)kHeads * kRow * 2, kHalfRope,
+                  kHeads, 1, CU_TENSOR_MAP_SWIZZLE_64B))
         return cudaErrorInvalidValue;
 
     cudaError_t e;
@@ -288,7 +305,6 @@ cudaError_t sm100_attend(const Problem& p, const void* q_hat, const CacheView& c
     a.plan = plan;
     a.seqlens = seqlens;
     a.q_len = p.q_len;
-    a.T_max = cache.T_max;
     a.scale_log2 = p.scale * 1.4426950408889634f;
     a.q_hat = (const __nv_bfloat16*)q_hat;
     a.o_lat = (__nv_bfloat16*)o_lat;
@@ -297,7 +313,7 @@ cudaError_t sm100_attend(const Problem& p, const void* q_hat, const CacheView& c
     a.status = status;
 
     if (events) events->record(MLA_EV_ATTEND_BEGIN, st);
-    e = launch_pdl(mla_attend_kernel, dim3(clusters * 2), dim3(kAttThreads), kAttSmem, st, 2, mC, a);
+    e = launch_pdl(mla_attend_kernel, dim3(clusters * 2), dim3(kAttThreads), kAttSmem, st, 2, mLat, mRope, mPf, mQR, a);
     if (e != cudaSuccess) return e;
     if (events) events->record(MLA_EV_ATTEND_END, st);
 

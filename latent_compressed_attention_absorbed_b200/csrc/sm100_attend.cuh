@@ -10,29 +10,38 @@
 // aggregate sum_j p_j c_KV,j before W_UV; m.lsln.cn section 2.1: softmax over
 // the whole history.)
 //
-// Work split.  A CTA owns 64 of the 128 heads of one query token and streams
-// full 576-wide cache tiles; the two CTAs of a head pair form one cluster so
-// that they run together and each tile is read from HBM once and served to
-// the other from L2.  Nothing is exchanged between CTAs.  Per CTA the fp32 accumulator is 64 heads x 512
-// latent columns: latent 0..255 lives in TMEM lanes 0..15 of each 32-lane
-// subpartition and latent 256..511 in lanes 16..31, both in columns 0..255
-// (M = 64 MMAs address either lane half).  Scores are split the same way:
-// the lower lane half accumulates S over latent 0..255 + RoPE 0..31, the
-// upper half over latent 256..511 + RoPE 32..63, and the two partial sums
-// of a row are added with one warp shuffle (lanes t and t+16 hold the same
-// head).
+// Work split.  The fp32 accumulator of 128 heads x 512 latent columns would
+// fill all 512 TMEM columns of an SM, and an M = 64 MMA runs at half the
+// tensor rate, so a CTA keeps all 128 heads (M = 128) and a cluster of two
+// CTAs splits the 576-wide cache row: CTA r loads and multiplies latent
+// columns 256r..256r+255 and RoPE columns 32r..32r+31 of every tile (the
+// cache crosses HBM and L2 once).  Each CTA computes a partial S over its
+// 288 columns, scales it to log2 units and rounds it to fp16; the pair swaps
+// the rounded partials through distributed shared memory (one bulk copy per
+// warp), both add the two halves (fp32 addition is commutative, so both CTAs
+// see the same S), run the same online softmax, and each accumulates its
+// 256 latent columns of O in TMEM.
 //
-// Scheduling (split-KV).  The unit of work is a query token (sequence b,
-// token i): it attends to keys 0..T_b-q_len+i, cut into 64-key tiles.  The
-// clusters divide the concatenated tile list of all units into equal
-// contiguous ranges (a fixed per-unit overhead is charged so tiny pieces are
-// avoided).  A unit processed by one cluster writes its normalised o_lat
-// directly (bf16); a unit cut across clusters writes fp32 partials plus a
-// base-2 LSE per head, merged by the combine kernel.
+// Scheduling (split-KV).  Sequences are cut into 64-key tiles.  The clusters
+// form groups of q_len (cluster c: group c / q_len, query token c % q_len);
+// the groups divide the concatenated tile list of all sequences into equal
+// contiguous ranges (a fixed per-sequence overhead is charged so tiny pieces
+// are avoided), and the q_len clusters of a group stream the same tiles at
+// the same time, so L2 serves the repeats.  A sequence processed by one
+// group writes its normalised o_lat directly (bf16); a sequence cut across
+// groups writes fp32 partials plus a base-2 LSE per head and token, merged by
+// the combine kernel.
 //
-// Roles per CTA (192 threads): warp 0 TMA producer, warp 1 TMEM owner and
-// MMA issuer, warps 2..5 softmax (warp w reads TMEM subpartition w%4: heads
-// 16*(w%4)..+15 in both lane halves).  Every wait is bounded; on expiry the
+// Roles per CTA (320 threads):
+//   warp 0     TMA producer (stage ring, L2 prefetch of the tiles ahead);
+//   warp 1     TMEM owner and MMA issuer (event loop: O as soon as P is
+//              published, S as soon as its tile and the S buffer are free);
+//   warps 2-5  softmax: add the two partial scores, online softmax, P into
+//              TMEM, rescale / normalise O, write o_lat or split partials;
+//   warps 6-9  exchange: read partial S out of TMEM, publish it (local copy
+//              for the softmax warps, bulk copy to the peer), load Q-hat.
+// Warp w reaches TMEM lanes 32*(w%4)..+31; lane l of warp w owns head
+// 32*(w%4)+l, a whole score row.  Every wait is bounded; on expiry the
 // kernel flags MLA_STATUS_TIMEOUT, stops issuing work and tears down
 // normally.
 #pragma once
@@ -46,57 +55,83 @@
 namespace mla {
 namespace sm100 {
 
-constexpr int kNk = 64;          // keys per tile
-constexpr int kHeads = 128;      // heads of a token
-constexpr int kRowsCta = 64;     // heads per CTA (M of every MMA)
-constexpr int kLat = 512;        // d_c
-constexpr int kRope = 64;        // d_r
+constexpr int kNk = 64;      // keys per tile
+constexpr int kHeads = 128;  // heads of a token (M of every MMA)
+constexpr int kLat = 512;    // d_c
+constexpr int kRope = 64;    // d_r
 constexpr int kRow = kLat + kRope;
 constexpr int kHalfLat = 256;
 constexpr int kHalfRope = 32;
 
-// Shared-memory map (offsets from a 1024-aligned base): a ring of full cache
-// tiles, each 9 SW128 chunks of 64 keys x 64 columns (8 latent, 1 RoPE).
-constexpr int kChunk = kNk * 128;                          // 8192
-constexpr int kTileBytes = 9 * kChunk;                     // 73728
-constexpr int kStages = 3;
-constexpr int kOffTiles = 0;
-constexpr int kOffBars = kOffTiles + kStages * kTileBytes;
+// Shared-memory map (offsets from a 1024-aligned base).
+//   stages: ring of this CTA's half tiles: 4 SW128 chunks of 64 keys x 64
+//           latent columns, then 64 keys x 32 RoPE columns (SW64);
+//   Own:    two buffers of this CTA's partial scores, 128 x 64 fp16 (rows of
+//           128 bytes, 16-byte chunks swizzled by row), read by the local
+//           softmax warps and bulk-copied to the peer's X buffer;
+//   X:      two buffers receiving the peer's partial scores (same layout);
+//   QR:     this CTA's RoPE half of Q-hat, 128 heads x 32 bf16 (SW64).
+constexpr int kChunk = kNk * 128;                     // 8192
+constexpr int kRopeChunk = kNk * 64;                  // 4096
+constexpr int kStageBytes = 4 * kChunk + kRopeChunk;  // 36864
+constexpr int kStages = 4;
+#ifndef MLA_PREFETCH_TILES
+#define MLA_PREFETCH_TILES 6
+#endif
+constexpr int kPrefetch = MLA_PREFETCH_TILES;  // tiles prefetched into L2 ahead of the stage loads
+constexpr int kXBytes = kHeads * 128;                 // 16384
+constexpr int kOffStages = 0;
+constexpr int kOffOwn = kOffStages + kStages * kStageBytes;
+constexpr int kOffX = kOffOwn + 2 * kXBytes;
+constexpr int kQRBytes = kHeads * 64;                  // 8192
+constexpr int kOffQR = kOffX + 2 * kXBytes;
+constexpr int kOffBars = kOffQR + kQRBytes;
 constexpr int kAttSmem = kOffBars + 256 + 1024;
-// Tensor-memory map: columns of 32 bits; lane half 0 = lanes 0..15 of each
-// subpartition, lane half 1 = lanes 16..31 (address lane field + 16).
+static_assert(kAttSmem <= 232448, "attention kernel shared memory exceeds 227 KB");
+
+// Tensor-memory map: 512 columns of 32 bits, lane = head.
 constexpr int kTmemCols = 512;
-constexpr uint32_t kLaneHalf1 = 16u << 16;
-constexpr int kTmemO = 0;      // O: half 0 latent 0..255, half 1 latent 256..511 (256 columns)
-constexpr int kTmemS = 256;    // S: half 0 partial over K-half a, half 1 over K-half b (64 columns)
-constexpr int kTmemP = 320;    // P: 64 bf16 probabilities, two per column, copied in both halves
-constexpr int kTmemQ = 352;    // Q-hat: half 0 latent 0..255 + RoPE 0..31, half 1 the rest (144 columns)
-constexpr int kAttThreads = 192;
+constexpr int kTmemO = 0;     // O: 256 fp32 latent columns of this CTA's half
+constexpr int kTmemS = 256;   // S: 64 fp32 partial scores
+constexpr int kTmemP = 320;   // P: two buffers of 64 bf16 probabilities, two per column
+constexpr int kTmemQ = 384;   // Q-hat latent half: 256 bf16, two per column (128 columns)
+constexpr int kAttThreads = 320;
 
 // Barrier indices (8 bytes each) inside the barrier block.
 enum {
     kBarFull0 = 0,
     kBarEmpty0 = kBarFull0 + kStages,
-    kBarQFull = kBarEmpty0 + kStages,
-    kBarSFull,
-    kBarSFree,
-    kBarPFull,
-    kBarPFree,
-    kBarOFull,
-    kBarOFree,
+    kBarQFull = kBarEmpty0 + kStages,  // Q-hat of the next piece loaded (4 exchange warps + RoPE-half TMA)
+    kBarSFull,                         // S(g) complete (MMA commit)
+    kBarSFree,                         // S(g) read out of TMEM (4 exchange warps)
+    kBarPFull0,                        // P(g) in TMEM buffer g%2 (4 softmax warps)
+    kBarPFree0 = kBarPFull0 + 2,       // O(g) complete: P buffer g%2 (and O) may be touched (MMA commit)
+    kBarOwnFull0 = kBarPFree0 + 2,     // own partial g in Own[g%2] (4 exchange warps)
+    kBarOwnFree0 = kBarOwnFull0 + 2,   // Own[g%2] read by the softmax warps (4)
+    kBarXFull0 = kBarOwnFree0 + 2,     // peer's partial g landed in X[g%2] (tx)
+    kBarXFree0 = kBarXFull0 + 2,       // the peer has read what we sent into its X[g%2] (4, remote)
+    kBarOFull = kBarXFree0 + 2,        // last O of a piece complete (MMA commit)
+    kBarOFree,                         // O read by the epilogue (4 softmax warps)
     kNumBars
 };
+static_assert(8 * (kNumBars + 2) <= 256, "barrier block too small");
 
-// Optional timing trace (compile with -DMLA_TRACE): clock64 stamps of the
-// first CTA at 16 fixed points of every tile, read back by mla_trace_read.
+// Optional timing trace (compile with -DMLA_TRACE): global-timer stamps (ns)
+// of both CTAs of one cluster at fixed points of every tile, read back by
+// mla_trace_read.  Events: 0 tile loads issued, 1 S issued, 2 O issued,
+// 3 S read by the exchange warps, 4 own partial published, 5 both partials
+// available to the softmax warps, 6 P published, 7 piece epilogue done,
+// 8 row max, 9 P computed, 10 tile data seen by the MMA warp, 11..13 P
+// published by warps 3, 4, 5.
 #ifdef MLA_TRACE
 #ifndef MLA_TRACE_CLUSTER
 #define MLA_TRACE_CLUSTER 0
 #endif
-__device__ unsigned long long g_mla_trace[4096][16];
-#define MLA_TRACE_POINT(ev, n)                                                                      \
-    do {                                                                                            \
-        if (cl == MLA_TRACE_CLUSTER && crank == 0 && (n) < 4096) g_mla_trace[(n)][(ev)] = clock64(); \
+constexpr int kTraceTiles = 4096;
+__device__ unsigned long long g_mla_trace[2][kTraceTiles][16];
+#define MLA_TRACE_POINT(ev, n)                                                                            \
+    do {                                                                                                  \
+        if (cl == MLA_TRACE_CLUSTER && (n) < kTraceTiles) g_mla_trace[r][(n)][(ev)] = global_timer_ns(); \
     } while (0)
 #else
 #define MLA_TRACE_POINT(ev, n) \
@@ -104,37 +139,38 @@ __device__ unsigned long long g_mla_trace[4096][16];
     } while (0)
 #endif
 
-// Scheduling plan written by the plan kernel into the workspace.
+// Scheduling plan written by the plan warp into the workspace.
 struct Plan {
-    int L;        // cost units per cluster
-    int ovh;      // cost charged per unit (query token)
-    int B;        // number of units = sequences x q_len
+    int L;        // cost units per group
+    int ovh;      // cost charged per sequence
+    int B;        // sequences
     int total;    // sum of costs
-    int n_split;  // units cut across clusters (listed after the prefix sums)
+    int n_split;  // sequences cut across groups (listed after the prefix sums)
     int q_len;
-    int pad[2];
-    // followed by int cost_prefix[B + 1], then int split_unit[B]
+    int groups;   // groups of q_len clusters
+    int pad;
+    // followed by int cost_prefix[B + 1], then int split_seq[B]
 };
 
 __device__ __forceinline__ const int* plan_prefix(const Plan* p) { return reinterpret_cast<const int*>(p + 1); }
 __device__ __forceinline__ const int* plan_splits(const Plan* p) { return plan_prefix(p) + p->B + 1; }
 
-// Tiles of unit b (0 if its sequence length was invalid).
+// Tiles of sequence b (0 if its length was invalid).
 __device__ __forceinline__ int plan_tiles(const int* pre, int b, int ovh) {
     const int c = pre[b + 1] - pre[b];
     return c > 0 ? c - ovh : 0;
 }
 
-// Segment iterator: the (unit, tile range) pieces of cluster `cl`.
+// Segment iterator: the (sequence, tile range) pieces of group `grp`.
 struct SegIter {
     const int* pre;
     int B, L, ovh, lo, hi, b;
-    __device__ void init(const Plan* plan, int cl) {
+    __device__ void init(const Plan* plan, int grp) {
         pre = plan_prefix(plan);
         B = plan->B;
         L = plan->L;
         ovh = plan->ovh;
-        lo = cl * L;
+        lo = grp * L;
         hi = lo + L;
         // largest b with pre[b] <= lo
         int a = 0, z = B;
@@ -164,13 +200,13 @@ struct SegIter {
     }
 };
 
-// Flat walk over the tiles of a cluster's pieces, with the piece's bounds.
+// Flat walk over the tiles of a group's pieces, with the piece's bounds.
 struct TileWalk {
     SegIter it;
     int seq, k0, k1, t, seg;
     bool whole, valid;
-    __device__ void init(const Plan* plan, int cl) {
-        it.init(plan, cl);
+    __device__ void init(const Plan* plan, int grp) {
+        it.init(plan, grp);
         seg = 0;
         valid = it.next(seq, k0, k1, whole);
         t = k0;
@@ -190,7 +226,6 @@ struct AttendArgs {
     const Plan* plan;
     const int32_t* seqlens;
     int q_len;
-    int T_max;
     float scale_log2;             // softmax_scale * log2(e)
     const __nv_bfloat16* q_hat;   // [B][q_len][128][576]
     __nv_bfloat16* o_lat;         // [B][q_len][128][512]
@@ -199,8 +234,19 @@ struct AttendArgs {
     int* status;
 };
 
+// Byte offset of 16-byte chunk c of row r in a buffer of 128-byte rows whose
+// chunks are permuted by row (c ^ (r % 8)), the SW128 pattern: the 8 rows a
+// quarter-warp touches at once land in 8 different bank groups.
+__device__ __forceinline__ uint32_t sw128(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
+
+// mapLat: cache [B][T_max][576] bf16, box 64 columns x 64 keys, SW128.
+// mapRope: same tensor, box 32 columns x 64 keys, SW64.
+// mapPf: the cache again, box 256 columns x 64 keys, no swizzle (L2 prefetch only).
+// mapQR: q_hat [U][128][576] bf16, box 32 columns x 128 heads, SW64.
 __global__ void __launch_bounds__(kAttThreads, 1)
-    mla_attend_kernel(const __grid_constant__ CUtensorMap mapCache, AttendArgs args) {
+    mla_attend_kernel(const __grid_constant__ CUtensorMap mapLat, const __grid_constant__ CUtensorMap mapRope,
+                      const __grid_constant__ CUtensorMap mapPf, const __grid_constant__ CUtensorMap mapQR,
+                      AttendArgs args) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -210,284 +256,411 @@ __global__ void __launch_bounds__(kAttThreads, 1)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(base_ptr + kOffBars + 8 * (kNumBars + 1));
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const uint32_t crank = cluster_ctarank();
-    const int hpart = crank & 1;       // heads 64*hpart .. +63
+    const uint32_t r = cluster_ctarank() & 1;  // latent half of this CTA
+    const uint32_t peer = r ^ 1;
     const int cl = (int)cluster_id_x();
     const int q_len = args.q_len;
-    if (threadIdx.x == 0) MLA_TRACE_POINT(0, 4095);
+    const int grp = cl / q_len, qi = cl % q_len;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(bar(kBarFull0 + s), 1);
             mbar_init(bar(kBarEmpty0 + s), 1);
         }
-        mbar_init(bar(kBarQFull), 4);
+        mbar_init(bar(kBarQFull), 5);
         mbar_init(bar(kBarSFull), 1);
         mbar_init(bar(kBarSFree), 4);
-        mbar_init(bar(kBarPFull), 4);
-        mbar_init(bar(kBarPFree), 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(bar(kBarPFull0 + s), 4);
+            mbar_init(bar(kBarPFree0 + s), 1);
+            mbar_init(bar(kBarOwnFull0 + s), 4);
+            mbar_init(bar(kBarOwnFree0 + s), 4);
+            mbar_init(bar(kBarXFull0 + s), 1);
+            mbar_init(bar(kBarXFree0 + s), 4);
+        }
         mbar_init(bar(kBarOFull), 1);
         mbar_init(bar(kBarOFree), 4);
         *abort_flag = 0;
         fence_mbar_init();
-        prefetch_tensormap(&mapCache);
+        prefetch_tensormap(&mapLat);
+        prefetch_tensormap(&mapRope);
+        prefetch_tensormap(&mapPf);
+        prefetch_tensormap(&mapQR);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
     }
     tc_fence_before();
-    __syncthreads();
+    // The peer's barriers must be initialised before any remote access.
+    cluster_sync();
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(base_ptr + kOffBars + 8 * kNumBars);
     // The set-up above overlaps the previous kernel; the plan, Q-hat and the
     // cache are read only once it has completed.
-    if (threadIdx.x == 0) MLA_TRACE_POINT(1, 4095);
     pdl_wait();
     if (threadIdx.x == 0) pdl_trigger();
-    if (threadIdx.x == 0) MLA_TRACE_POINT(2, 4095);
+    const bool active = grp < args.plan->groups;
+    const int quarter = warp & 3;
+    const int m = quarter * 32 + lane;                          // head / TMEM lane (warps 2..9)
+    const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;  // the warp's TMEM subpartition
 
-    if (warp == 0) {
+    if (!active) {
+        // idle cluster (the cluster count is not a multiple of q_len)
+    } else if (warp == 0) {
         // ======================================================== TMA producer (runs up to kStages tiles ahead)
+        // Tiles kPrefetch ahead of the loads are prefetched into L2, so that a
+        // stage, once freed, refills at L2 rather than HBM latency.
         if (lane == 0) {
-            TileWalk w;
-            w.init(args.plan, cl);
+            TileWalk w, wp;
+            w.init(args.plan, grp);
+            wp = w;
+            for (int i = 0; i < kPrefetch && wp.valid; ++i) {
+                tma_prefetch_3d(&mapPf, kHalfLat * r, wp.t * kNk, wp.seq);
+                tma_prefetch_3d(&mapRope, kLat + kHalfRope * r, wp.t * kNk, wp.seq);
+                wp.advance();
+            }
             for (int n = 0; w.valid && !*abort_flag; ++n, w.advance()) {
+                if (kPrefetch > 0 && wp.valid) {
+                    tma_prefetch_3d(&mapPf, kHalfLat * r, wp.t * kNk, wp.seq);
+                    tma_prefetch_3d(&mapRope, kLat + kHalfRope * r, wp.t * kNk, wp.seq);
+                    wp.advance();
+                }
                 const int st = n % kStages;
                 if (n >= kStages && !mbar_wait(bar(kBarEmpty0 + st), ((n / kStages) - 1) & 1)) {
                     *abort_flag = 1;
                     break;
                 }
-                const uint32_t dst = base + kOffTiles + st * kTileBytes;
-                mbar_arrive_expect_tx(bar(kBarFull0 + st), kTileBytes);
-                for (int c = 0; c < 9; ++c)
-                    tma_load_3d(dst + c * kChunk, &mapCache, bar(kBarFull0 + st), 64 * c, w.t * kNk, w.seq / q_len);
+                const uint32_t dst = base + kOffStages + st * kStageBytes;
+                mbar_arrive_expect_tx(bar(kBarFull0 + st), kStageBytes);
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    tma_load_3d(dst + c * kChunk, &mapLat, bar(kBarFull0 + st), kHalfLat * r + 64 * c, w.t * kNk, w.seq);
+                tma_load_3d(dst + 4 * kChunk, &mapRope, bar(kBarFull0 + st), kLat + kHalfRope * r, w.t * kNk, w.seq);
                 MLA_TRACE_POINT(0, n);
             }
         }
     } else if (warp == 1) {
-        // ======================================================== MMA issuer (whole warp waits, lane 0 issues)
-        constexpr uint32_t idS = idesc_bf16_f32(kRowsCta, kNk, false, false);
-        constexpr uint32_t idO = idesc_bf16_f32(kRowsCta, kHalfLat, false, true);
-        bool ok = true;
-        // O(g) += P(g) . C(g) for both latent halves; the first K-step overwrites O at the start of a piece.
-        auto issue_O = [&](int g, bool first_in_seg, bool last_in_seg) {
-            const uint64_t dO = smem_desc(base + kOffTiles + (g % kStages) * kTileBytes, kChunk, 1024, kSw128);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const uint32_t acc = (!first_in_seg || k > 0) ? 1u : 0u;
-                mma_f16_ts(tmem + kTmemO, tmem + kTmemP + 8 * k, dO + ((2048 * k) >> 4), idO, acc);
-                mma_f16_ts(tmem + kLaneHalf1 + kTmemO, tmem + kLaneHalf1 + kTmemP + 8 * k,
-                           dO + ((4 * kChunk + 2048 * k) >> 4), idO, acc);
-            }
-            mma_commit(bar(kBarPFree));
-            mma_commit(bar(kBarEmpty0 + (g % kStages)));
-            if (last_in_seg) mma_commit(bar(kBarOFull));
+        // ======================================================== MMA issuer (whole warp polls, lane 0 issues)
+        constexpr uint32_t idS = idesc_bf16_f32(kHeads, kNk, false, false);
+        constexpr uint32_t idO = idesc_bf16_f32(kHeads, kHalfLat, false, true);
+        const uint32_t stages = base + kOffStages;
+        // Descriptor templates: the start-address field (bits 0..13, address >> 4)
+        // is advanced by adding byte offsets >> 4.
+        const uint64_t dLatK = smem_desc(stages, 16, 1024, kSw128);       // cache latent, K-major (S)
+        const uint64_t dRopeK = smem_desc(stages, 16, 512, kSw64);        // cache RoPE, K-major (S)
+        const uint64_t dLatMN = smem_desc(stages, kChunk, 1024, kSw128);  // cache latent, MN-major (O)
+        const uint64_t dQR = smem_desc(base + kOffQR, 16, 512, kSw64);    // Q-hat RoPE half (S, A operand)
+        TileWalk ws, wo;  // next tile whose S / O is issued
+        ws.init(args.plan, grp);
+        wo = ws;
+        int gs = 0, go = 0;
+        int T_s = ws.valid ? args.seqlens[ws.seq] : 0;  // length of the sequence of tile gs
+        // Warp-uniform non-blocking barrier probe (lane 0 decides).
+        auto ready = [&](uint32_t b, uint32_t parity) -> bool {
+            return __shfl_sync(0xffffffffu, mbar_test_wait(b, parity) ? 1 : 0, 0) != 0;
         };
-        TileWalk w;
-        w.init(args.plan, cl);
-        bool prev_first = false, prev_last = false, prev_pending = false;
-        int prev_seg = 0;
-        int g = 0;
-        // O(g-1) normally follows S(g) so that S(g) overlaps the softmax of
-        // tile g-1; at the end of a piece it goes first, because the softmax
-        // warps load the next piece's Q-hat only after that piece's epilogue.
-        auto finish_prev = [&]() -> bool {
-            if (!mbar_wait(bar(kBarPFull), (g - 1) & 1)) return false;
-            if (prev_first && prev_seg > 0 && !mbar_wait(bar(kBarOFree), (prev_seg - 1) & 1)) return false;
+        // O += P(g) . cache latent half(g); the first tile of a piece overwrites
+        // O (after the previous piece's epilogue has read it).
+        auto o_ready = [&]() -> bool {
+            if (!wo.valid || !ready(bar(kBarPFull0 + (go & 1)), (go >> 1) & 1)) return false;
+            return !(wo.first() && wo.seg > 0) || ready(bar(kBarOFree), (wo.seg - 1) & 1);
+        };
+        auto issue_O = [&]() {
+            const int g = go;
+            const bool first = wo.first(), last = wo.last();
             tc_fence_after();
-            MLA_TRACE_POINT(4, g - 1);
-            if (lane == 0) issue_O(g - 1, prev_first, prev_last);
-            __syncwarp();
-            MLA_TRACE_POINT(5, g - 1);
-            prev_pending = false;
-            return true;
-        };
-        // Descriptor templates: start-address field (bits 0..13, address >> 4)
-        // is advanced by adding byte offsets >> 4 to one base descriptor.
-        const uint64_t dS0 = smem_desc(base + kOffTiles, 16, 1024, kSw128);
-        const uint64_t dO0 = smem_desc(base + kOffTiles, kChunk, 1024, kSw128);
-        int T_b = 0;
-        for (; w.valid && ok && !*abort_flag; ++g, w.advance()) {
-            if (prev_pending && prev_last && !finish_prev()) { ok = false; break; }
-            if (w.first()) {
-                T_b = args.seqlens[w.seq / q_len];
-                if (!mbar_wait(bar(kBarQFull), w.seg & 1)) { ok = false; break; }
+            if (lane == 0) {
+                MLA_TRACE_POINT(15, g);
+                const int st = g % kStages;
+                const uint64_t dB = dLatMN + ((kOffStages + st * kStageBytes) >> 4);
+                const uint32_t pA = tmem + kTmemP + 32 * (g & 1);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    mma_f16_ts(tmem + kTmemO, pA + 8 * k, dB + ((2048 * k) >> 4), idO, (!first || k > 0) ? 1u : 0u);
+                mma_commit(bar(kBarPFree0 + (g & 1)));
+                mma_commit(bar(kBarEmpty0 + st));
+                if (last) mma_commit(bar(kBarOFull));
+                MLA_TRACE_POINT(2, g);
             }
-            const int st = g % kStages;
-            const uint32_t tile_off = kOffTiles + st * kTileBytes;
-            const uint32_t tile = base + tile_off;
-            if (!mbar_wait(bar(kBarFull0 + st), (g / kStages) & 1)) { ok = false; break; }
-            MLA_TRACE_POINT(1, g);
-            const int valid = T_b - w.t * kNk;
+            __syncwarp();
+            ++go;
+            wo.advance();
+        };
+        // S(g) = Q-hat half . cache half^T over this CTA's 288 columns: it needs
+        // the piece's Q-hat, the tile, and S(g-1) read out of TMEM.
+        auto s_ready = [&]() -> bool {
+            const int g = gs;
+            if (!ws.valid) return false;
+            if (ws.first() && !ready(bar(kBarQFull), ws.seg & 1)) return false;
+            if (!ready(bar(kBarFull0 + g % kStages), (g / kStages) & 1)) return false;
+#ifdef MLA_TRACE
+            if (lane == 0 && g < kTraceTiles && g_mla_trace[r][g][10] == 0 && cl == MLA_TRACE_CLUSTER)
+                MLA_TRACE_POINT(10, g);
+#endif
+            return g == 0 || ready(bar(kBarSFree), (g - 1) & 1);
+        };
+        // The 18 MMAs of S go out in three groups; a pending O is issued between
+        // groups (issuing runs at the tensor pipe's pace), so O(g) never waits
+        // for a whole S.
+        auto issue_S = [&]() {
+            const int g = gs;
+            const uint32_t tile_off = kOffStages + (g % kStages) * kStageBytes;
+            const int valid = T_s - ws.t * kNk;
             if (valid < kNk) {
-                // Rows at or beyond T_b hold no cached token: zero them so that
-                // masked (p = 0) rows cannot inject NaN/Inf into P.C.
+                // Rows at or beyond T_b hold no cached token: zero the latent
+                // part so that masked (p = 0) rows cannot inject NaN/Inf into P.C.
                 const int r0 = valid < 0 ? 0 : valid;
-                for (int r = r0 + (lane >> 3); r < kNk; r += 4)
-                    for (int c = 0; c < 9; ++c) st_shared_v4(tile + c * kChunk + r * 128 + (lane & 7) * 16, 0, 0, 0, 0);
+                for (int row = r0 + (lane >> 3); row < kNk; row += 4)
+                    for (int c = 0; c < 4; ++c)
+                        st_shared_v4(base + tile_off + c * kChunk + row * 128 + (lane & 7) * 16, 0, 0, 0, 0);
                 fence_proxy_async_smem();
             }
             __syncwarp();
-            // S(g) reuses the S columns: the softmax warps must have read S(g-1).
-            if (g > 0 && !mbar_wait(bar(kBarSFree), (g - 1) & 1)) { ok = false; break; }
             tc_fence_after();
-            MLA_TRACE_POINT(2, g);
-            if (lane == 0) {
-                // half a: latent chunks 0..3 then RoPE columns 0..31; half b: chunks 4..7 then RoPE 32..63
-                const uint64_t dS = dS0 + ((tile_off) >> 4);
+            const uint32_t dS = tmem + kTmemS;
+            const uint64_t dL = dLatK + (tile_off >> 4);
+            if (lane == 0) MLA_TRACE_POINT(14, g);
 #pragma unroll
-                for (int kk = 0; kk < 18; ++kk) {
-                    const uint32_t oa = kk < 16 ? (kk / 4) * kChunk + 32 * (kk % 4) : 8 * kChunk + 32 * (kk - 16);
-                    const uint32_t ob = kk < 16 ? (4 + kk / 4) * kChunk + 32 * (kk % 4) : 8 * kChunk + 64 + 32 * (kk - 16);
-                    mma_f16_ts(tmem + kTmemS, tmem + kTmemQ + 8 * kk, dS + (oa >> 4), idS, kk ? 1u : 0u);
-                    mma_f16_ts(tmem + kLaneHalf1 + kTmemS, tmem + kLaneHalf1 + kTmemQ + 8 * kk, dS + (ob >> 4), idS,
-                               kk ? 1u : 0u);
+            for (int grp6 = 0; grp6 < 3; ++grp6) {
+                if (lane == 0) {
+#pragma unroll
+                    for (int kk = 0; kk < 6; ++kk) {
+                        const int k = 6 * grp6 + kk;
+                        if (k < 16) {
+                            mma_f16_ts(dS, tmem + kTmemQ + 8 * k, dL + (((k >> 2) * kChunk + 32 * (k & 3)) >> 4),
+                                       idS, k ? 1u : 0u);
+                        } else {
+                            const int j = k - 16;
+                            mma_f16_ss(dS, dQR + ((32 * j) >> 4), dRopeK + ((tile_off + 4 * kChunk + 32 * j) >> 4),
+                                       idS, 1u);
+                        }
+                    }
+                    if (grp6 == 2) {
+                        mma_commit(bar(kBarSFull));
+                        MLA_TRACE_POINT(1, g);
+                    }
                 }
-                mma_commit(bar(kBarSFull));
+                __syncwarp();
+                if (grp6 < 2 && o_ready()) issue_O();
             }
-            __syncwarp();
-            MLA_TRACE_POINT(3, g);
-            if (prev_pending && !finish_prev()) { ok = false; break; }
-            prev_first = w.first();
-            prev_last = w.last();
-            prev_seg = w.seg;
-            prev_pending = true;
+            ++gs;
+            const int seq_before = ws.seq;
+            ws.advance();
+            if (ws.valid && ws.seq != seq_before) T_s = args.seqlens[ws.seq];
+        };
+        // Event loop: O first (it frees a stage and a P buffer), then S.  Every
+        // dependency of an S or O points to earlier tiles, so polling both
+        // cannot deadlock.
+        bool ok = true;
+        uint64_t t_idle = 0;
+        while (wo.valid && !*abort_flag) {
+            bool progress = false;
+            if (o_ready()) {
+                issue_O();
+                progress = true;
+            } else if (s_ready()) {
+                issue_S();
+                progress = true;
+            }
+            if (progress) {
+                t_idle = 0;
+            } else if (t_idle == 0) {
+                t_idle = global_timer_ns();
+            } else if (global_timer_ns() - t_idle > MLA_WAIT_LIMIT_NS) {
+                ok = false;
+                break;
+            }
         }
-        if (ok && !*abort_flag && prev_pending && !finish_prev()) ok = false;
+        if (!ok) *abort_flag = 1;
+    } else if (warp >= 6) {
+        // ======================================================== exchange warps 6..9
+        const float sl2 = args.scale_log2;
+        const uint32_t x_peer = mapa(base + kOffX, peer);
+        const uint32_t xfull_peer = mapa(bar(kBarXFull0), peer);
+        bool ok = true;
+        // Q-hat of unit u, this CTA's half: row m's 256 latent values -> TMEM
+        // (this thread), the 128 x 32 RoPE block -> shared memory by TMA
+        // (issued by thread 192).
+        auto load_q = [&](int u) {
+            if (threadIdx.x == 192) {
+                mbar_arrive_expect_tx(bar(kBarQFull), kQRBytes);
+                tma_load_3d(base + kOffQR, &mapQR, bar(kBarQFull), kLat + kHalfRope * r, 0, u);
+            }
+            const uint4* src = reinterpret_cast<const uint4*>(args.q_hat + ((size_t)u * kHeads + m) * kRow) + 32 * r;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint4 x[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) x[j] = __ldg(src + 8 * c + j);
+                uint32_t v[32];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    v[4 * j] = x[j].x; v[4 * j + 1] = x[j].y; v[4 * j + 2] = x[j].z; v[4 * j + 3] = x[j].w;
+                }
+                tmem_st32(tmem + lane_addr + kTmemQ + 32 * c, v);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(kBarQFull));
+        };
+        TileWalk w;
+        w.init(args.plan, grp);
+        if (w.valid) load_q(w.seq * q_len + qi);
+        for (int h = 0; w.valid && ok && !*abort_flag; ++h, w.advance()) {
+            const int hb = h & 1;
+            // ---- partial S(h) of this half, in log2 units, rounded to fp16
+            if (!mbar_wait(bar(kBarSFull), h & 1)) { ok = false; break; }
+            tc_fence_after();
+            uint32_t own[32];
+            {
+                uint32_t va[32], vb[32];
+                tmem_ld32(tmem + lane_addr + kTmemS, va);
+                tmem_ld32(tmem + lane_addr + kTmemS + 32, vb);
+                tmem_wait_ld();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(kBarSFree));
+                if (threadIdx.x == 192) MLA_TRACE_POINT(3, h);
+                // S(h) was the last reader of this piece's Q-hat: load the next piece's.
+                if (w.last()) {
+                    TileWalk nx = w;
+                    nx.advance();
+                    if (nx.valid) load_q(nx.seq * q_len + qi);
+                }
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    own[j] = pack_f16(__uint_as_float(va[2 * j]) * sl2, __uint_as_float(va[2 * j + 1]) * sl2);
+                    own[16 + j] = pack_f16(__uint_as_float(vb[2 * j]) * sl2, __uint_as_float(vb[2 * j + 1]) * sl2);
+                }
+            }
+            // ---- publish: Own[hb] (read by our softmax warps and by the bulk copy
+            // into the peer's X[hb]); both readers of tile h-2 must be done.
+            if (h >= 2) {
+                if (!mbar_wait(bar(kBarOwnFree0 + hb), ((h >> 1) - 1) & 1)) { ok = false; break; }
+#ifndef MLA_NO_XCHG
+                if (!mbar_wait_cluster(bar(kBarXFree0 + hb), ((h >> 1) - 1) & 1)) { ok = false; break; }
+#endif
+            }
+            const uint32_t own_buf = base + kOffOwn + hb * kXBytes;
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                st_shared_v4(own_buf + sw128(m, c), own[4 * c], own[4 * c + 1], own[4 * c + 2], own[4 * c + 3]);
+#ifdef MLA_XCHG_STASYNC
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                st_async_v4_b32(x_peer + hb * kXBytes + sw128(m, c), own[4 * c], own[4 * c + 1], own[4 * c + 2],
+                                own[4 * c + 3], xfull_peer + 8 * hb);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(kBarOwnFull0 + hb));
+#elif defined(MLA_NO_XCHG)
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(kBarOwnFull0 + hb));
+#else
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                const uint32_t off = quarter * 32 * 128;
+                bulk_copy_s2s(x_peer + hb * kXBytes + off, own_buf + off, 32 * 128, xfull_peer + 8 * hb);
+                mbar_arrive(bar(kBarOwnFull0 + hb));
+            }
+#endif
+            // The peer's partial for tile h lands in our X[hb] (its phase h/2).
+            if (threadIdx.x == 192) {
+#ifndef MLA_NO_XCHG
+                mbar_arrive_expect_tx(bar(kBarXFull0 + hb), kXBytes);
+#endif
+                MLA_TRACE_POINT(4, h);
+            }
+        }
         if (!ok) *abort_flag = 1;
     } else {
         // ======================================================== softmax warps 2..5
-        // Thread (quarter, lane): head row m = 16*quarter + lane%16 of this CTA,
-        // lane half lh = lane/16: it reads the lh partial scores, handles keys
-        // 32*lh..32*lh+31 of the row, and owns latent half lh of O.
-        const int quarter = warp & 3;
-        const int lh = lane >> 4;
-        const int m = quarter * 16 + (lane & 15);
-        const int head = hpart * kRowsCta + m;
-        const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;  // the warp's subpartition
-        const float sl2 = args.scale_log2;
+        const uint32_t xfree_peer = mapa(bar(kBarXFree0), peer);
         bool ok = true;
         TileWalk w;
-        w.init(args.plan, cl);
+        w.init(args.plan, grp);
         float m_used = -CUDART_INF_F, l_sum = 0.f;
         int n_keys = 0;
         for (int g = 0; w.valid && ok && !*abort_flag; ++g, w.advance()) {
-            if (w.first()) {
-                // Q-hat row `head`, K-half lh -> TMEM (S(g-1), the last reader of the old Q-hat, has completed).
-                const int u = w.seq;
-                const uint4* src = reinterpret_cast<const uint4*>(args.q_hat + ((size_t)u * kHeads + head) * kRow);
-                // 36 loads of 16 bytes in two batches (latent 0..127 | latent 128..255 + RoPE)
-                {
-                    uint4 x[16];
+            const int b2 = g & 1;
+            // ---- S(g) = own partial + the peer's, added in the same order on both CTAs
+            if (!mbar_wait(bar(kBarOwnFull0 + b2), (g >> 1) & 1)) { ok = false; break; }
+#ifndef MLA_NO_XCHG
+            if (!mbar_wait_cluster(bar(kBarXFull0 + b2), (g >> 1) & 1)) { ok = false; break; }
+#endif
+            float s[kNk];
+            {
+                const uint32_t own_buf = base + kOffOwn + b2 * kXBytes;
+#ifdef MLA_NO_XCHG
+                const uint32_t x_buf = own_buf;
+#else
+                const uint32_t x_buf = base + kOffX + b2 * kXBytes;
+#endif
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) x[j] = __ldg(src + lh * 32 + j);
+                for (int c = 0; c < 8; ++c) {
+                    uint32_t a0, a1, a2, a3, o0, o1, o2, o3;
+                    ld_shared_v4u(own_buf + sw128(m, c), a0, a1, a2, a3);
+                    ld_shared_v4u(x_buf + sw128(m, c), o0, o1, o2, o3);
+                    const uint32_t mine[4] = {a0, a1, a2, a3};
+                    const uint32_t oth[4] = {o0, o1, o2, o3};
 #pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        uint32_t v[32];
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            v[4 * j] = x[8 * c + j].x; v[4 * j + 1] = x[8 * c + j].y;
-                            v[4 * j + 2] = x[8 * c + j].z; v[4 * j + 3] = x[8 * c + j].w;
-                        }
-                        tmem_st32(tmem + lane_addr + kTmemQ + 32 * c, v);
+                    for (int q = 0; q < 4; ++q) {
+                        const float2 v = sum_f16x2(mine[q], oth[q]);
+                        s[8 * c + 2 * q] = v.x;
+                        s[8 * c + 2 * q + 1] = v.y;
                     }
                 }
-                {
-                    uint4 x[20];
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) x[j] = __ldg(src + lh * 32 + 16 + j);
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) x[16 + j] = __ldg(src + 64 + lh * 4 + j);
-#pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        uint32_t v[32];
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            v[4 * j] = x[8 * c + j].x; v[4 * j + 1] = x[8 * c + j].y;
-                            v[4 * j + 2] = x[8 * c + j].z; v[4 * j + 3] = x[8 * c + j].w;
-                        }
-                        tmem_st32(tmem + lane_addr + kTmemQ + 64 + 32 * c, v);
-                    }
-                    uint32_t v[16];
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        v[4 * j] = x[16 + j].x; v[4 * j + 1] = x[16 + j].y;
-                        v[4 * j + 2] = x[16 + j].z; v[4 * j + 3] = x[16 + j].w;
-                    }
-                    tmem_st16(tmem + lane_addr + kTmemQ + 128, v);
-                }
-                tmem_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(kBarQFull));
-                if (threadIdx.x == 64) MLA_TRACE_POINT(7, 4095);
             }
-            // ---- partial S(g) of this lane half
-            if (!mbar_wait(bar(kBarSFull), g & 1)) { ok = false; break; }
-            tc_fence_after();
-            MLA_TRACE_POINT(7, g);
-            uint32_t va[32], vb[32];
-            tmem_ld32(tmem + lane_addr + kTmemS, va);
-            tmem_ld32(tmem + lane_addr + kTmemS + 32, vb);
-            tmem_wait_ld();
-            tc_fence_before();
+            // Both buffers are consumed (their values are in registers and used
+            // by the adds above), so relaxed arrives suffice.
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(kBarSFree));
-            // ---- full scores of keys 32*lh .. +31: own partial + the other half's (lane ^ 16)
-            float s[32];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const float give = __uint_as_float(lh ? va[j] : vb[j]);  // the half the partner scores
-                const float mine = __uint_as_float(lh ? vb[j] : va[j]);
-                const float other = __shfl_xor_sync(0xffffffffu, give, 16);
-                s[j] = (mine + other) * sl2;
+            if (lane == 0) {
+                mbar_arrive(bar(kBarOwnFree0 + b2));
+#ifndef MLA_NO_XCHG
+                mbar_arrive_remote_relaxed(xfree_peer + 8 * b2);
+#endif
             }
-            // unit u = (b, i) sees keys 0..T_b-q_len+i
-            if (w.first()) n_keys = args.seqlens[w.seq / q_len] - q_len + 1 + w.seq % q_len;
-            const int key0 = w.t * kNk + 32 * lh;
-            if (key0 + 32 > n_keys) {
+            if (threadIdx.x == 64) MLA_TRACE_POINT(5, g);
+            // ---- online softmax in base 2, lazy rescaling of O
+            // query token qi of sequence b sees keys 0..T_b-q_len+qi
+            if (w.first()) n_keys = args.seqlens[w.seq] - q_len + 1 + qi;
+            const int key0 = w.t * kNk;
+            if (key0 + kNk > n_keys) {
 #pragma unroll
-                for (int j = 0; j < 32; ++j)
+                for (int j = 0; j < kNk; ++j)
                     if (key0 + j >= n_keys) s[j] = -CUDART_INF_F;
             }
             float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
 #pragma unroll
-            for (int j = 4; j < 32; j += 4) {
+            for (int j = 4; j < kNk; j += 4) {
                 mx0 = fmaxf(mx0, s[j]); mx1 = fmaxf(mx1, s[j + 1]);
                 mx2 = fmaxf(mx2, s[j + 2]); mx3 = fmaxf(mx3, s[j + 3]);
             }
-            float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+            const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+            if (threadIdx.x == 64) MLA_TRACE_POINT(8, g);
             const bool first = w.first();
             const bool grow = mx > m_used + 8.0f;  // rescale only when the max grows by > 2^8
             const float mb_new = grow ? mx : m_used;
             const float mb = (mb_new == -CUDART_INF_F) ? 0.f : mb_new;
-            uint32_t own[16];
+            uint32_t pk[32];
             float rs0 = 0.f, rs1 = 0.f;
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
+            for (int j = 0; j < 32; ++j) {
                 const float p0 = ex2(s[2 * j] - mb), p1 = ex2(s[2 * j + 1] - mb);
                 rs0 += p0;
                 rs1 += p1;
-                own[j] = pack_bf16(p0, p1);
+                pk[j] = pack_bf16(p0, p1);
             }
-            float rs = rs0 + rs1;
-            rs += __shfl_xor_sync(0xffffffffu, rs, 16);
-            uint32_t pk[32];
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const uint32_t oth = __shfl_xor_sync(0xffffffffu, own[j], 16);
-                pk[j] = lh ? oth : own[j];
-                pk[16 + j] = lh ? own[j] : oth;
-            }
-            MLA_TRACE_POINT(11, g);
-            // P(g) overwrites P(g-1) and a rescale touches O: wait for O += P(g-1) C(g-1).
-            if (g > 0 && !mbar_wait(bar(kBarPFree), (g - 1) & 1)) { ok = false; break; }
-            tc_fence_after();
-            MLA_TRACE_POINT(12, g);
+            if (threadIdx.x == 64) MLA_TRACE_POINT(9, g);
+            // P buffer b2 was last read by O(g-2).
+            if (g >= 2 && !mbar_wait(bar(kBarPFree0 + b2), ((g >> 1) - 1) & 1)) { ok = false; break; }
             if (grow) {
                 if (!first) {
+                    // O must hold everything up to tile g-1 before it is rescaled.
+                    if (!mbar_wait(bar(kBarPFree0 + (b2 ^ 1)), ((g - 1) >> 1) & 1)) { ok = false; break; }
+                    tc_fence_after();
                     const float f = ex2(m_used - mx);
                     l_sum *= f;
 #pragma unroll 1
@@ -502,22 +675,25 @@ __global__ void __launch_bounds__(kAttThreads, 1)
                 }
                 m_used = mx;
             }
-            l_sum += rs;
-            tmem_st32(tmem + lane_addr + kTmemP, pk);
+            tc_fence_after();
+            l_sum += rs0 + rs1;
+            tmem_st32(tmem + lane_addr + kTmemP + 32 * b2, pk);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(kBarPFull));
-            MLA_TRACE_POINT(13, g);
-            // ---- epilogue at the end of a piece: this thread owns O row m, latent half lh
+            if (lane == 0) mbar_arrive(bar(kBarPFull0 + b2));
+            if (threadIdx.x == 64) MLA_TRACE_POINT(6, g);
+            if (threadIdx.x == 96) MLA_TRACE_POINT(11, g);
+            if (threadIdx.x == 128) MLA_TRACE_POINT(12, g);
+            if (threadIdx.x == 160) MLA_TRACE_POINT(13, g);
+            // ---- epilogue at the end of a piece: this thread owns O row m (256 columns)
             if (w.last()) {
                 if (!mbar_wait(bar(kBarOFull), w.seg & 1)) { ok = false; break; }
                 tc_fence_after();
-                if (threadIdx.x == 64) MLA_TRACE_POINT(5, 4095);
                 const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
-                const int u = w.seq;
+                const int u = w.seq * q_len + qi;
                 if (w.whole) {
-                    __nv_bfloat16* dst = args.o_lat + ((size_t)u * kHeads + head) * kLat + lh * kHalfLat;
+                    __nv_bfloat16* dst = args.o_lat + ((size_t)u * kHeads + m) * kLat + r * kHalfLat;
 #pragma unroll 1
                     for (int c0 = 0; c0 < kHalfLat; c0 += 32) {
                         uint32_t v[32];
@@ -534,30 +710,29 @@ __global__ void __launch_bounds__(kAttThreads, 1)
                         }
                     }
                 } else {
-                    // fp32 partial, head-minor: [slot][col4][head][4] so that the 16 lanes of
-                    // a half warp (16 consecutive heads) write 256 contiguous bytes per store.
-                    const int slot = cl + u;
-                    float4* dst = reinterpret_cast<float4*>(args.part_o) + (size_t)slot * (kLat / 4) * kHeads + head;
+                    // fp32 partial, head-minor: [slot][col4][head][4], so that a warp
+                    // (32 consecutive heads) writes 512 contiguous bytes per store.
+                    const size_t slot = (size_t)(grp + w.seq) * q_len + qi;
+                    float4* dst = reinterpret_cast<float4*>(args.part_o) + slot * (kLat / 4) * kHeads + m;
 #pragma unroll 1
                     for (int c0 = 0; c0 < kHalfLat; c0 += 32) {
                         uint32_t v[32];
                         tmem_ld32(tmem + lane_addr + kTmemO + c0, v);
                         tmem_wait_ld();
-                        const int k0 = (lh * kHalfLat + c0) / 4;
+                        const int k0 = (r * kHalfLat + c0) / 4;
 #pragma unroll
                         for (int j = 0; j < 32; j += 4)
                             dst[(size_t)(k0 + j / 4) * kHeads] =
                                 make_float4(__uint_as_float(v[j]) * inv, __uint_as_float(v[j + 1]) * inv,
                                             __uint_as_float(v[j + 2]) * inv, __uint_as_float(v[j + 3]) * inv);
                     }
-                    if (lh == 0)
-                        args.part_lse[(size_t)slot * kHeads + head] =
-                            l_sum > 0.f ? m_used + __log2f(l_sum) : -CUDART_INF_F;
+                    if (r == 0)
+                        args.part_lse[slot * kHeads + m] = l_sum > 0.f ? m_used + __log2f(l_sum) : -CUDART_INF_F;
                 }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(kBarOFree));
-                if (threadIdx.x == 64) MLA_TRACE_POINT(6, 4095);
+                if (threadIdx.x == 64) MLA_TRACE_POINT(7, g);
                 m_used = -CUDART_INF_F;
                 l_sum = 0.f;
             }
@@ -566,37 +741,36 @@ __global__ void __launch_bounds__(kAttThreads, 1)
     }
 
     if (*abort_flag && threadIdx.x == 0) atomicOr(args.status, MLA_STATUS_TIMEOUT);
-    if (threadIdx.x == 64) MLA_TRACE_POINT(3, 4095);
     tc_fence_before();
     __syncthreads();
     if (warp == 1) tmem_dealloc(tmem, kTmemCols);
-    if (threadIdx.x == 32) MLA_TRACE_POINT(4, 4095);
+    // The peer may still copy scores into this CTA's shared memory or arrive
+    // on its barriers: neither CTA leaves before both are done.
+    cluster_sync();
 }
 
 // ------------------------------------------------------------------ plan
 
-// cost_b = ceil(T_b / 64) + ovh (0 for an invalid length); prefix sums and the
-// per-cluster share L = ceil(total / clusters), at least min_units; the list
-// of sequences cut across clusters; o_lat = 0 for sequences with an invalid
-// length (their decode has no defined result).  One warp.
+// Per sequence: cost_b = ceil(T_b / 64) + ovh (0 for an invalid length);
+// prefix sums, the per-group share L = ceil(total / groups) (at least
+// min_units), the list of sequences cut across groups, and o_lat = 0 for the
+// tokens of sequences with an invalid length (their decode has no defined
+// result).  One warp.
 __device__ __forceinline__ void mla_plan_warp(const int32_t* __restrict__ seqlens, int B, int q_len, int T_max,
                                               int clusters, int ovh, int min_units, Plan* plan, int* status,
                                               __nv_bfloat16* o_lat, int lane) {
-    const int U = B * q_len;
     int* pre = reinterpret_cast<int*>(plan + 1);
-    int* splits = pre + U + 1;
+    int* splits = pre + B + 1;
+    const int groups = clusters / q_len > 0 ? clusters / q_len : 1;
     int carry = 0;
     if (lane == 0) pre[0] = 0;
-    for (int base = 0; base < U; base += 32) {
-        const int u = base + lane;
+    for (int base = 0; base < B; base += 32) {
+        const int b = base + lane;
         int c = 0;
-        if (u < U) {
-            const int T = seqlens[u / q_len];
-            if (T < q_len || T > T_max) {
-                if (u % q_len == 0) atomicOr(status, MLA_STATUS_BAD_SEQLEN);
-            } else {
-                c = (T - q_len + 1 + u % q_len + kNk - 1) / kNk + ovh;
-            }
+        if (b < B) {
+            const int T = seqlens[b];
+            if (T < q_len || T > T_max) atomicOr(status, MLA_STATUS_BAD_SEQLEN);
+            else c = (T + kNk - 1) / kNk + ovh;
         }
         int v = c;
 #pragma unroll
@@ -604,40 +778,41 @@ __device__ __forceinline__ void mla_plan_warp(const int32_t* __restrict__ seqlen
             const int y = __shfl_up_sync(0xffffffffu, v, o);
             if (lane >= o) v += y;
         }
-        if (u < U) pre[u + 1] = carry + v;
+        if (b < B) pre[b + 1] = carry + v;
         carry += __shfl_sync(0xffffffffu, v, 31);
     }
-    int L = (carry + clusters - 1) / clusters;
+    int L = (carry + groups - 1) / groups;
     if (L < min_units) L = min_units;
     if (L < 1) L = 1;
     __syncwarp();
     int n_split = 0;
-    for (int base = 0; base < U; base += 32) {
-        const int u = base + lane;
+    for (int base = 0; base < B; base += 32) {
+        const int b = base + lane;
         bool split = false, invalid = false;
-        if (u < U) {
-            const int lo = pre[u], hi = pre[u + 1];
+        if (b < B) {
+            const int lo = pre[b], hi = pre[b + 1];
             if (hi == lo) invalid = true;
             else split = (lo + ovh) / L != (hi - 1) / L;
         }
-        const unsigned m = __ballot_sync(0xffffffffu, split);
-        if (split) splits[n_split + __popc(m & ((1u << lane) - 1))] = u;
-        n_split += __popc(m);
+        const unsigned msk = __ballot_sync(0xffffffffu, split);
+        if (split) splits[n_split + __popc(msk & ((1u << lane) - 1))] = b;
+        n_split += __popc(msk);
         unsigned inv = __ballot_sync(0xffffffffu, invalid);
         while (inv) {
-            const int ui = base + __ffs(inv) - 1;
+            const int bi = base + __ffs(inv) - 1;
             inv &= inv - 1;
-            uint4* dst = reinterpret_cast<uint4*>(o_lat + (size_t)ui * kHeads * kLat);
-            for (int i = lane; i < kHeads * kLat / 8; i += 32) dst[i] = make_uint4(0, 0, 0, 0);
+            uint4* dst = reinterpret_cast<uint4*>(o_lat + (size_t)bi * q_len * kHeads * kLat);
+            for (int i = lane; i < q_len * kHeads * kLat / 8; i += 32) dst[i] = make_uint4(0, 0, 0, 0);
         }
     }
     if (lane == 0) {
         plan->L = L;
         plan->ovh = ovh;
-        plan->B = U;
+        plan->B = B;
         plan->total = carry;
         plan->n_split = n_split;
         plan->q_len = q_len;
+        plan->groups = groups;
     }
 }
 
@@ -657,8 +832,9 @@ __global__ void __launch_bounds__(32) mla_plan_kernel(const int32_t* __restrict_
 // contiguous 2 KiB of the head-minor partials.  A CTA covers KPC column
 // quads; its G groups take every G-th piece and keep a running (max, sum,
 // accumulator) each, merged through shared memory at the end.  G = 1 suits
-// batches whose units are cut into a few pieces; G = 8 gives small batches
-// (a unit cut into tens of pieces) enough loads in flight.
+// batches whose sequences are cut into a few pieces; G = 8 gives small
+// batches (a sequence cut into tens of pieces) enough loads in flight.
+// A split unit is (split sequence, query token): blockIdx / per-unit CTAs.
 template <int G, int KPC>
 __global__ void __launch_bounds__(128 * G * KPC) mla_combine_kernel(const Plan* __restrict__ plan,
                                                                     const float* __restrict__ part_o,
@@ -670,20 +846,23 @@ __global__ void __launch_bounds__(128 * G * KPC) mla_combine_kernel(const Plan* 
     __shared__ float2 s_mw[G > 1 ? G : 1][KPC][kHeads];
     pdl_wait();
     pdl_trigger();
+    const int q_len = plan->q_len;
     const int work = blockIdx.x / kPerUnit;
-    if (work >= plan->n_split) return;
+    if (work >= plan->n_split * q_len) return;
     const int h = threadIdx.x % kHeads;
     const int kk = (threadIdx.x / kHeads) % KPC;
     const int g = threadIdx.x / (kHeads * KPC);
     const int k = (blockIdx.x % kPerUnit) * KPC + kk;  // column quad
-    const int u = plan_splits(plan)[work];
+    const int b = plan_splits(plan)[work / q_len];
+    const int qi = work % q_len;
+    const int u = b * q_len + qi;
     const int* pre = plan_prefix(plan);
     const int L = plan->L, ovh = plan->ovh;
-    const int tiles = plan_tiles(pre, u, ovh);
-    const int c_lo = pre[u], c_hi = pre[u + 1];
+    const int tiles = plan_tiles(pre, b, ovh);
+    const int c_lo = pre[b], c_hi = pre[b + 1];
     const int p_lo = c_lo / L, p_hi = (c_hi - 1) / L;
-    // Cluster p holds tiles [p L - c_lo - ovh, (p+1) L - c_lo - ovh) of the
-    // unit, clipped to [0, tiles); an empty clip wrote no partial.
+    // Group p holds tiles [p L - c_lo - ovh, (p+1) L - c_lo - ovh) of the
+    // sequence, clipped to [0, tiles); an empty clip wrote no partial.
     auto nonempty = [&](int p) {
         int s0 = p * L - c_lo - ovh, e0 = (p + 1) * L - c_lo - ovh;
         s0 = s0 < 0 ? 0 : (s0 > tiles ? tiles : s0);
@@ -702,7 +881,7 @@ __global__ void __launch_bounds__(128 * G * KPC) mla_combine_kernel(const Plan* 
             lse[j] = -CUDART_INF_F;
             v[j] = make_float4(0.f, 0.f, 0.f, 0.f);
             if (p <= p_hi && nonempty(p)) {
-                const size_t slot = (size_t)(p + u);
+                const size_t slot = (size_t)(p + b) * q_len + qi;
                 lse[j] = __ldg(part_lse + slot * kHeads + h);
                 v[j] = __ldg(po + slot * (kLat / 4) * kHeads);
             }
@@ -711,20 +890,20 @@ __global__ void __launch_bounds__(128 * G * KPC) mla_combine_kernel(const Plan* 
 #pragma unroll
         for (int j = 0; j < kBatch; ++j) mb = fmaxf(mb, lse[j]);
         if (mb == -CUDART_INF_F) continue;  // nothing but empty pieces so far
-        const float r = exp2f(m - mb);      // m = -inf gives 0
-        wsum *= r;
-        acc.x *= r;
-        acc.y *= r;
-        acc.z *= r;
-        acc.w *= r;
+        const float rr = exp2f(m - mb);     // m = -inf gives 0
+        wsum *= rr;
+        acc.x *= rr;
+        acc.y *= rr;
+        acc.z *= rr;
+        acc.w *= rr;
 #pragma unroll
         for (int j = 0; j < kBatch; ++j) {
-            const float w = exp2f(lse[j] - mb);  // empty piece: 2^-inf = 0
-            wsum += w;
-            acc.x += w * v[j].x;
-            acc.y += w * v[j].y;
-            acc.z += w * v[j].z;
-            acc.w += w * v[j].w;
+            const float wgt = exp2f(lse[j] - mb);  // empty piece: 2^-inf = 0
+            wsum += wgt;
+            acc.x += wgt * v[j].x;
+            acc.y += wgt * v[j].y;
+            acc.z += wgt * v[j].z;
+            acc.w += wgt * v[j].w;
         }
         m = mb;
     }

@@ -42,6 +42,12 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
 }
 
+// Arrive on an mbarrier of another CTA of the cluster (address from mapa),
+// relaxed: for signals whose prior reads have already been consumed.
+__device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t cluster_bar) {
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
+}
+
 // Arrive on an mbarrier of another CTA of the cluster (address from mapa).
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_bar) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
@@ -52,6 +58,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Non-blocking probe: true if the phase with this parity has completed.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
         : "r"(bar), "r"(parity)
@@ -146,6 +165,17 @@ __device__ __forceinline__ void st_async_v4_b32(uint32_t cluster_addr, uint32_t 
         : "memory");
 }
 
+// Bulk copy from this CTA's shared memory to another CTA's (addresses from
+// mapa), completing `bytes` of transaction count on that CTA's mbarrier.
+// Addresses 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_copy_s2s(uint32_t dst_cluster, uint32_t src, uint32_t bytes,
+                                              uint32_t cluster_bar) {
+    asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     dst_cluster),
+                 "r"(src), "r"(bytes), "r"(cluster_bar)
+                 : "memory");
+}
+
 // 16-byte load from another CTA's shared memory (address from mapa).
 __device__ __forceinline__ void ld_cluster_v4u(uint32_t cluster_addr, uint32_t& a, uint32_t& b, uint32_t& c,
                                                uint32_t& d) {
@@ -172,6 +202,14 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
         "[%2];" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
         : "memory");
+}
+
+// Prefetch a tile of a tensor into L2 (no shared memory, no completion).
+__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* map, int c0, int c1, int c2) {
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(c0), "r"(c1), "r"(c2)
+                 : "memory");
 }
 
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
@@ -326,6 +364,19 @@ __device__ __forceinline__ float2 unpack_f16(uint32_t v) {
         : "r"(v));
     return r;
 }
+// Two fp16 pairs added in fp32: (a.lo + b.lo, a.hi + b.hi), each half
+// widened exactly (mixed-precision adds, no separate conversions).
+__device__ __forceinline__ float2 sum_f16x2(uint32_t a, uint32_t b) {
+    float2 r;
+    asm("{\n\t.reg .f16 al, ah, bl, bh;\n\t.reg .f32 t0, t1;\n\t"
+        "mov.b32 {al, ah}, %2;\n\tmov.b32 {bl, bh}, %3;\n\t"
+        "add.rn.f32.f16 t0, al, 0f00000000;\n\tadd.rn.f32.f16 t1, ah, 0f00000000;\n\t"
+        "add.rn.f32.f16 %0, bl, t0;\n\tadd.rn.f32.f16 %1, bh, t1;\n\t}"
+        : "=f"(r.x), "=f"(r.y)
+        : "r"(a), "r"(b));
+    return r;
+}
+
 __device__ __forceinline__ void ld_shared_v4u(uint32_t addr, uint32_t& a, uint32_t& b, uint32_t& c, uint32_t& d) {
     asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(a), "=r"(b), "=r"(c), "=r"(d) : "r"(addr)
                  : "memory");
