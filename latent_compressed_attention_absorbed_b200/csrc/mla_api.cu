@@ -101,7 +101,7 @@ int choose_path(const Problem& p, int q_len, const mla_decode_opts_t* o, bool* f
     if (want == 1 && !can)
         return fail(MLA_ERR_UNSUPPORTED,
                     "the sm_100a path needs a compute-capability 10.0 device, bf16, H=128, d_c=512, d_r=64, "
-                    "d_n=128, d_v=128 and q_len <= 4");
+                    "d_n=128, d_v=128 and q_len <= 16");
     *fast = (want == 1) || (want == 0 && can);
     t_path = *fast ? "sm100" : "generic";
     return MLA_OK;
@@ -111,6 +111,17 @@ int pairs_for(const mla_decode_opts_t* o) {
     int n = (o && o->num_pairs > 0) ? o->num_pairs : sm100_default_pairs();
     if (n > 1024) n = 1024;  // the split combine handles at most 1024 pieces per sequence
     return n > 0 ? n : 1;
+}
+
+// The kernels store 32-byte vectors into the workspace; its base is rounded up
+// to 256 bytes inside the caller's buffer (mla_workspace_bytes includes the
+// slack), so any 16-byte-aligned buffer of that size works.
+constexpr size_t kWsAlign = 256;
+void* align_ws(void* ws, size_t* bytes) {
+    const uintptr_t p = reinterpret_cast<uintptr_t>(ws);
+    const uintptr_t a = (p + kWsAlign - 1) & ~uintptr_t(kWsAlign - 1);
+    *bytes = (a - p) > *bytes ? 0 : *bytes - (a - p);
+    return reinterpret_cast<void*>(a);
 }
 
 struct DecodeLayout {
@@ -207,9 +218,9 @@ size_t mla_workspace_bytes(const mla_dims_t* dims, int32_t B, int32_t q_len) {
     p.q_len = q_len;
     const bool fast = sm100_supported(p, q_len);
     const DecodeLayout g = decode_layout(p, false, 1);
-    if (!fast) return g.total;
+    if (!fast) return g.total + kWsAlign;
     const DecodeLayout f = decode_layout(p, true, sm100_default_pairs());
-    return f.total > g.total ? f.total : g.total;
+    return (f.total > g.total ? f.total : g.total) + kWsAlign;
 }
 
 int mla_absorb_query(const mla_dims_t* dims, const void* q_nope, const void* q_rope, const void* W_UK,
@@ -258,10 +269,11 @@ int mla_attend_latent(const mla_dims_t* dims, const void* q_hat, const mla_cache
     cudaError_t e;
     if (fast) {
         const int pairs = pairs_for(opts);
-        const size_t need = sm100_attend_workspace_bytes(p, pairs);
+        const size_t need = sm100_attend_workspace_bytes(p, pairs) + kWsAlign;
         if (!workspace || workspace_bytes < need || !aligned16(workspace))
             return fail(MLA_ERR_WORKSPACE, "attend workspace needs %zu bytes (16-byte aligned), got %zu", need,
                         workspace_bytes);
+        workspace = align_ws(workspace, &workspace_bytes);
         e = sm100_attend(p, q_hat, cv, seqlens, o_lat, workspace, workspace_bytes, pairs,
                          opts ? opts->overhead_tiles : -1, opts ? opts->min_tiles : 0, status, (cudaStream_t)stream);
     } else {
@@ -313,9 +325,10 @@ int mla_decode_ex(const mla_dims_t* dims, const void* q_nope, const void* q_rope
     if (rc) return rc;
     const int pairs = fast ? pairs_for(opts) : 1;
     const DecodeLayout L = decode_layout(p, fast, pairs);
-    if (!workspace || workspace_bytes < L.total || !aligned16(workspace))
-        return fail(MLA_ERR_WORKSPACE, "decode workspace needs %zu bytes (16-byte aligned), got %zu", L.total,
-                    workspace_bytes);
+    if (!workspace || workspace_bytes < L.total + kWsAlign || !aligned16(workspace))
+        return fail(MLA_ERR_WORKSPACE, "decode workspace needs %zu bytes (16-byte aligned), got %zu",
+                    L.total + kWsAlign, workspace_bytes);
+    workspace = align_ws(workspace, &workspace_bytes);
     int* status = device_status_ptr();
     if (!status) return fail(MLA_ERR_CUDA, "no CUDA device / status word");
     char* ws = static_cast<char*>(workspace);
@@ -337,14 +350,18 @@ int mla_decode_ex(const mla_dims_t* dims, const void* q_nope, const void* q_rope
         pr.clusters = pairs;
         pr.overhead_tiles = opts ? opts->overhead_tiles : -1;
         pr.min_tiles = opts ? opts->min_tiles : 0;
-        e = sm100_absorb(p, q_nope, q_rope, W_UK, seqlens, q_hat, st, &pr);
+        const bool small = B * q_len <= kSmallRows;
+        e = B * q_len <= kSmallAbsorbRows ? sm100_absorb_small(p, q_nope, q_rope, W_UK, seqlens, q_hat, st, &pr)
+                                          : sm100_absorb(p, q_nope, q_rope, W_UK, seqlens, q_hat, st, &pr);
         ev.record(MLA_EV_ABSORB_DONE, st);
         if (e == cudaSuccess)
             e = sm100_attend(p, q_hat, cv, seqlens, o_lat, ws + L.attend, L.total - L.attend, pairs,
                              opts ? opts->overhead_tiles : -1, opts ? opts->min_tiles : 0, status, st, &ev,
-                             /*plan_ready=*/true);
+                             /*plan_ready=*/true, /*combine=*/!small);
         ev.record(MLA_EV_COMBINE_DONE, st);
-        if (e == cudaSuccess) e = sm100_project(p, o_lat, W_UV, B * q_len, out, st);
+        if (e == cudaSuccess)
+            e = small ? sm100_project_small(p, ws + L.attend, pairs, o_lat, W_UV, out, st)
+                      : sm100_project(p, o_lat, W_UV, B * q_len, out, st);
     } else {
         e = generic_absorb(p, q_nope, q_rope, W_UK, seqlens, q_hat, st);
         ev.record(MLA_EV_ABSORB_DONE, st);

@@ -85,9 +85,19 @@ cudaError_t sm100_absorb(const Problem& p, const void* q_nope, const void* q_rop
 cudaError_t sm100_attend(const Problem& p, const void* q_hat, const CacheView& cache, const int32_t* seqlens,
                          void* o_lat, void* workspace, size_t ws_bytes, int num_pairs, int overhead_tiles,
                          int min_tiles, int* status, cudaStream_t st, const Events* events = nullptr,
-                         bool plan_ready = false);
+                         bool plan_ready = false, bool combine = true);
 cudaError_t sm100_project(const Problem& p, const void* o_lat, const void* W_UV, int rows, void* out,
                           cudaStream_t st);
+// Small batches: matrix-vector kernels.  The project step (B * q_len <= 8)
+// reads the attention workspace and merges split partials itself (the
+// attention step then runs without its combine kernel); the absorb step
+// uses them up to 2 rows, the tensor-core GEMM above.
+constexpr int kSmallRows = 8;
+constexpr int kSmallAbsorbRows = 2;
+cudaError_t sm100_absorb_small(const Problem& p, const void* q_nope, const void* q_rope, const void* W_UK,
+                               const int32_t* seqlens, void* q_hat, cudaStream_t st, const PlanRequest* plan);
+cudaError_t sm100_project_small(const Problem& p, void* attend_workspace, int num_pairs, const void* o_lat,
+                                const void* W_UV, void* out, cudaStream_t st);
 size_t sm100_attend_workspace_bytes(const Problem& p, int num_pairs);
 int sm100_default_pairs();
 

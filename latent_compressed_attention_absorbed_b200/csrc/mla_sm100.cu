@@ -12,6 +12,7 @@
 #include "mla_rope.cuh"
 #include "sm100_attend.cuh"
 #include "sm100_gemm.cuh"
+#include "sm100_gemv.cuh"
 
 #ifdef MLA_TRACE
 // Copies the attention kernel's timing trace (4096 tiles x 16 stamps) to host
@@ -107,6 +108,7 @@ cudaError_t set_smem(K kernel, int bytes, bool (&done)[kMaxDev]) {
     return e;
 }
 bool g_smem_absorb[kMaxDev], g_smem_project[kMaxDev], g_smem_attend[kMaxDev];
+bool g_smem_absorb_gemv[4][kMaxDev], g_smem_project_gemv[4][kMaxDev];
 
 // Launch with programmatic dependent launch allowed: the kernel may start
 // while the previous kernel on the stream is finishing; it calls
@@ -142,7 +144,7 @@ constexpr int kAbsorbStages = 2;
 // else the batch rounded up to 16 (the MMA still computes 128 rows; the rows
 // past the batch are never stored).
 int plan_ovh(int overhead_tiles) { return overhead_tiles < 0 ? 2 : overhead_tiles; }
-int plan_min_units(int min_tiles) { return min_tiles > 0 ? min_tiles : 1; }
+int plan_min_units(int min_tiles) { return min_tiles > 0 ? min_tiles : 2; }
 int gemm_a_rows(int rows) { return rows >= 128 ? 128 : ((rows + 15) / 16) * 16; }
 constexpr int kProjStages = 4;
 constexpr int kProjNT = 64;
@@ -245,6 +247,55 @@ cudaError_t sm100_project(const Problem& p, const void* o_lat, const void* W_UV,
     return launch_pdl(kern, grid, dim3(128), Cfg::kSmem, st, 1, mA, mB, a);
 }
 
+// Small batches (rows <= kGemvMaxRows): CUDA-core matrix-vector kernels with
+// the weight slices staged in shared memory; R = rows rounded up to 1, 2, 4, 8.
+template <int R>
+static cudaError_t absorb_gemv_launch(const AbsorbGemvArgs& a, cudaStream_t st) {
+    static_assert(R == 1 || R == 2 || R == 4 || R == 8, "row count");
+    constexpr int idx = R == 1 ? 0 : R == 2 ? 1 : R == 4 ? 2 : 3;
+    cudaError_t e = set_smem(absorb_gemv_kernel<R>, absorb_gemv_smem<R>(), g_smem_absorb_gemv[idx]);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(absorb_gemv_kernel<R>, dim3(kHeads + 1, 2), dim3(128), absorb_gemv_smem<R>(), st, 1, a);
+}
+template <int R>
+static cudaError_t project_gemv_launch(const ProjectGemvArgs& a, cudaStream_t st) {
+    constexpr int idx = R == 1 ? 0 : R == 2 ? 1 : R == 4 ? 2 : 3;
+    cudaError_t e = set_smem(project_gemv_kernel<R>, project_gemv_smem<R>(), g_smem_project_gemv[idx]);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(project_gemv_kernel<R>, dim3(kHeads), dim3(512), project_gemv_smem<R>(), st, 1, a);
+}
+
+cudaError_t sm100_absorb_small(const Problem& p, const void* q_nope, const void* q_rope, const void* W_UK,
+                               const int32_t* seqlens, void* q_hat, cudaStream_t st, const PlanRequest* plan) {
+    const int rows = p.B * p.q_len;
+    if (rows < 1 || rows > kGemvMaxRows) return cudaErrorInvalidValue;
+    AbsorbGemvArgs a;
+    memset(&a, 0, sizeof(a));
+    a.q_nope = (const __nv_bfloat16*)q_nope;
+    a.q_rope = (const __nv_bfloat16*)q_rope;
+    a.W_UK = (const __nv_bfloat16*)W_UK;
+    a.seqlens = seqlens;
+    a.rows = rows;
+    a.q_len = p.q_len;
+    a.q_hat = (__nv_bfloat16*)q_hat;
+    a.rope = p.rope;
+    a.status = device_status_ptr();
+    a.plan = nullptr;
+    if (plan) {
+        a.plan = static_cast<Plan*>(plan->plan);
+        a.plan_B = p.B;
+        a.plan_T_max = plan->T_max;
+        a.plan_clusters = plan->clusters;
+        a.plan_ovh = plan_ovh(plan->overhead_tiles);
+        a.plan_min_units = plan_min_units(plan->min_tiles);
+        a.plan_olat = static_cast<__nv_bfloat16*>(plan->o_lat);
+    }
+    if (rows == 1) return absorb_gemv_launch<1>(a, st);
+    if (rows == 2) return absorb_gemv_launch<2>(a, st);
+    if (rows <= 4) return absorb_gemv_launch<4>(a, st);
+    return absorb_gemv_launch<8>(a, st);
+}
+
 // Clusters of the attention grid: at least one per query token (a group of
 // q_len clusters streams one sequence piece, one cluster per token).
 static int attend_clusters(int pairs, int q_len) { return pairs < q_len ? q_len : pairs; }
@@ -272,7 +323,8 @@ size_t sm100_attend_workspace_bytes(const Problem& p, int num_pairs) {
 
 cudaError_t sm100_attend(const Problem& p, const void* q_hat, const CacheView& cache, const int32_t* seqlens,
                          void* o_lat, void* workspace, size_t ws_bytes, int num_pairs, int overhead_tiles,
-                         int min_tiles, int* status, cudaStream_t st, const Events* events, bool plan_ready) {
+                         int min_tiles, int* status, cudaStream_t st, const Events* events, bool plan_ready,
+                         bool combine) {
     const int clusters = attend_clusters(num_pairs, p.q_len);
     size_t off_part, off_lse;
     const size_t need = attend_layout(p, clusters, &off_part, &off_lse);
@@ -308,6 +360,7 @@ cudaError_t sm100_attend(const Problem& p, const void* q_hat, const CacheView& c
     a.scale_log2 = p.scale * 1.4426950408889634f;
     a.q_hat = (const __nv_bfloat16*)q_hat;
     a.o_lat = (__nv_bfloat16*)o_lat;
+    a.o_lat_v8 = (reinterpret_cast<uintptr_t>(o_lat) & 31u) == 0;
     a.part_o = reinterpret_cast<float*>(ws + off_part);
     a.part_lse = reinterpret_cast<float*>(ws + off_lse);
     a.status = status;
@@ -317,22 +370,36 @@ cudaError_t sm100_attend(const Problem& p, const void* q_hat, const CacheView& c
     if (e != cudaSuccess) return e;
     if (events) events->record(MLA_EV_ATTEND_END, st);
 
-    // Split units number at most min(B * q_len, clusters - 1).  With many
-    // pieces per unit (small batches) the warp-per-piece merge is used.
+    // Split units number at most min(B * q_len, clusters); one CTA covers
+    // eight heads of one unit.
     const int units = p.B * p.q_len;
     const int max_split = units < clusters ? units : clusters;
-    const Plan* cplan = plan;
-    const float* po = a.part_o;
-    const float* pl = a.part_lse;
-    __nv_bfloat16* ol = (__nv_bfloat16*)o_lat;
-    if (4 * units < clusters)
-        e = launch_pdl(mla_combine_kernel<8, 1>, dim3(max_split * (kLat / 4)), dim3(1024), 0, st, 1, cplan, po, pl,
-                       ol);
-    else
-        e = launch_pdl(mla_combine_kernel<1, 2>, dim3(max_split * (kLat / 8)), dim3(256), 0, st, 1, cplan, po, pl,
-                       ol);
+    if (combine)
+        e = launch_pdl(mla_combine_kernel, dim3(max_split * (kHeads / 8)), dim3(256), 0, st, 1, (const Plan*)plan,
+                       (const float*)a.part_o, (const float*)a.part_lse, (__nv_bfloat16*)o_lat);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
+}
+
+cudaError_t sm100_project_small(const Problem& p, void* attend_workspace, int num_pairs, const void* o_lat,
+                                const void* W_UV, void* out, cudaStream_t st) {
+    const int rows = p.B * p.q_len;
+    if (rows < 1 || rows > kGemvMaxRows) return cudaErrorInvalidValue;
+    size_t off_part, off_lse;
+    attend_layout(p, num_pairs, &off_part, &off_lse);
+    char* ws = static_cast<char*>(attend_workspace);
+    ProjectGemvArgs a;
+    a.plan = reinterpret_cast<const Plan*>(ws);
+    a.o_lat = (const __nv_bfloat16*)o_lat;
+    a.part_o = reinterpret_cast<const float*>(ws + off_part);
+    a.part_lse = reinterpret_cast<const float*>(ws + off_lse);
+    a.W_UV = (const __nv_bfloat16*)W_UV;
+    a.rows = rows;
+    a.out = (__nv_bfloat16*)out;
+    if (rows == 1) return project_gemv_launch<1>(a, st);
+    if (rows == 2) return project_gemv_launch<2>(a, st);
+    if (rows <= 4) return project_gemv_launch<4>(a, st);
+    return project_gemv_launch<8>(a, st);
 }
 
 }  // namespace mla

@@ -128,6 +128,7 @@ static_assert(8 * (kNumBars + 2) <= 256, "barrier block too small");
 #define MLA_TRACE_CLUSTER 0
 #endif
 constexpr int kTraceTiles = 4096;
+constexpr int kTraceProlog = kTraceTiles - 1;  // row of kernel-level stamps
 __device__ unsigned long long g_mla_trace[2][kTraceTiles][16];
 #define MLA_TRACE_POINT(ev, n)                                                                            \
     do {                                                                                                  \
@@ -138,6 +139,9 @@ __device__ unsigned long long g_mla_trace[2][kTraceTiles][16];
     do {                       \
     } while (0)
 #endif
+// Kernel-level stamps (row kTraceProlog): 0 entry, 1 after set-up, 2 after the
+// grid dependency wait, 3 first Q-hat loaded, 4 epilogue start, 5 epilogue
+// end, 6 teardown start, 7 exit.
 
 // Scheduling plan written by the plan warp into the workspace.
 struct Plan {
@@ -229,7 +233,8 @@ struct AttendArgs {
     float scale_log2;             // softmax_scale * log2(e)
     const __nv_bfloat16* q_hat;   // [B][q_len][128][576]
     __nv_bfloat16* o_lat;         // [B][q_len][128][512]
-    float* part_o;                // [slots][128 col4][128 heads][4]
+    int o_lat_v8;                 // o_lat is 32-byte aligned: 32-byte stores
+    float* part_o;                // [slots][64 column octets][128 heads][8]
     float* part_lse;              // [slots][128]
     int* status;
 };
@@ -262,6 +267,7 @@ __global__ void __launch_bounds__(kAttThreads, 1)
     const int q_len = args.q_len;
     const int grp = cl / q_len, qi = cl % q_len;
 
+    if (threadIdx.x == 0) MLA_TRACE_POINT(0, kTraceProlog);
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(bar(kBarFull0 + s), 1);
@@ -295,11 +301,13 @@ __global__ void __launch_bounds__(kAttThreads, 1)
     // The peer's barriers must be initialised before any remote access.
     cluster_sync();
     tc_fence_after();
+    if (threadIdx.x == 0) MLA_TRACE_POINT(1, kTraceProlog);
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(base_ptr + kOffBars + 8 * kNumBars);
     // The set-up above overlaps the previous kernel; the plan, Q-hat and the
     // cache are read only once it has completed.
     pdl_wait();
     if (threadIdx.x == 0) pdl_trigger();
+    if (threadIdx.x == 0) MLA_TRACE_POINT(2, kTraceProlog);
     const bool active = grp < args.plan->groups;
     const int quarter = warp & 3;
     const int m = quarter * 32 + lane;                          // head / TMEM lane (warps 2..9)
@@ -489,16 +497,20 @@ __global__ void __launch_bounds__(kAttThreads, 1)
             }
             const uint4* src = reinterpret_cast<const uint4*>(args.q_hat + ((size_t)u * kHeads + m) * kRow) + 32 * r;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint4 x[8];
+            for (int half = 0; half < 2; ++half) {
+                uint4 x[16];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) x[j] = __ldg(src + 8 * c + j);
-                uint32_t v[32];
+                for (int j = 0; j < 16; ++j) x[j] = __ldg(src + 16 * half + j);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    v[4 * j] = x[j].x; v[4 * j + 1] = x[j].y; v[4 * j + 2] = x[j].z; v[4 * j + 3] = x[j].w;
+                for (int c = 0; c < 2; ++c) {
+                    uint32_t v[32];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        v[4 * j] = x[8 * c + j].x; v[4 * j + 1] = x[8 * c + j].y;
+                        v[4 * j + 2] = x[8 * c + j].z; v[4 * j + 3] = x[8 * c + j].w;
+                    }
+                    tmem_st32(tmem + lane_addr + kTmemQ + 64 * half + 32 * c, v);
                 }
-                tmem_st32(tmem + lane_addr + kTmemQ + 32 * c, v);
             }
             tmem_wait_st();
             tc_fence_before();
@@ -508,6 +520,7 @@ __global__ void __launch_bounds__(kAttThreads, 1)
         TileWalk w;
         w.init(args.plan, grp);
         if (w.valid) load_q(w.seq * q_len + qi);
+        if (threadIdx.x == 192) MLA_TRACE_POINT(3, kTraceProlog);
         for (int h = 0; w.valid && ok && !*abort_flag; ++h, w.advance()) {
             const int hb = h & 1;
             // ---- partial S(h) of this half, in log2 units, rounded to fp16
@@ -690,6 +703,7 @@ __global__ void __launch_bounds__(kAttThreads, 1)
             if (w.last()) {
                 if (!mbar_wait(bar(kBarOFull), w.seg & 1)) { ok = false; break; }
                 tc_fence_after();
+                if (threadIdx.x == 64) MLA_TRACE_POINT(4, kTraceProlog);
                 const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
                 const int u = w.seq * q_len + qi;
                 if (w.whole) {
@@ -700,31 +714,40 @@ __global__ void __launch_bounds__(kAttThreads, 1)
                         tmem_ld32(tmem + lane_addr + kTmemO + c0, v);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int j = 0; j < 32; j += 8) {
-                            uint4 o;
-                            o.x = pack_bf16(__uint_as_float(v[j]) * inv, __uint_as_float(v[j + 1]) * inv);
-                            o.y = pack_bf16(__uint_as_float(v[j + 2]) * inv, __uint_as_float(v[j + 3]) * inv);
-                            o.z = pack_bf16(__uint_as_float(v[j + 4]) * inv, __uint_as_float(v[j + 5]) * inv);
-                            o.w = pack_bf16(__uint_as_float(v[j + 6]) * inv, __uint_as_float(v[j + 7]) * inv);
-                            *reinterpret_cast<uint4*>(dst + c0 + j) = o;
+                        for (int j = 0; j < 32; j += 16) {
+                            uint32_t o[8];
+#pragma unroll
+                            for (int q = 0; q < 8; ++q)
+                                o[q] = pack_bf16(__uint_as_float(v[j + 2 * q]) * inv, __uint_as_float(v[j + 2 * q + 1]) * inv);
+                            if (args.o_lat_v8) {
+                                st_global_v8(dst + c0 + j, o[0], o[1], o[2], o[3], o[4], o[5], o[6], o[7]);
+                            } else {
+                                *reinterpret_cast<uint4*>(dst + c0 + j) = make_uint4(o[0], o[1], o[2], o[3]);
+                                *reinterpret_cast<uint4*>(dst + c0 + j + 8) = make_uint4(o[4], o[5], o[6], o[7]);
+                            }
                         }
                     }
                 } else {
-                    // fp32 partial, head-minor: [slot][col4][head][4], so that a warp
-                    // (32 consecutive heads) writes 512 contiguous bytes per store.
+                    // fp32 partial in column octets, [slot][c8][head][8]: a warp (32
+                    // consecutive heads) writes 1 KB contiguous per octet (one 32-byte
+                    // store per lane), and a consumer reading one head gets whole
+                    // 32-byte sectors.
                     const size_t slot = (size_t)(grp + w.seq) * q_len + qi;
-                    float4* dst = reinterpret_cast<float4*>(args.part_o) + slot * (kLat / 4) * kHeads + m;
+                    float* dst = args.part_o + (slot * (kLat / 8) * kHeads + m) * 8;
 #pragma unroll 1
                     for (int c0 = 0; c0 < kHalfLat; c0 += 32) {
                         uint32_t v[32];
                         tmem_ld32(tmem + lane_addr + kTmemO + c0, v);
                         tmem_wait_ld();
-                        const int k0 = (r * kHalfLat + c0) / 4;
+                        const int o0 = (r * kHalfLat + c0) / 8;
 #pragma unroll
-                        for (int j = 0; j < 32; j += 4)
-                            dst[(size_t)(k0 + j / 4) * kHeads] =
-                                make_float4(__uint_as_float(v[j]) * inv, __uint_as_float(v[j + 1]) * inv,
-                                            __uint_as_float(v[j + 2]) * inv, __uint_as_float(v[j + 3]) * inv);
+                        for (int j = 0; j < 32; j += 8) {
+                            uint32_t o[8];
+#pragma unroll
+                            for (int q = 0; q < 8; ++q) o[q] = __float_as_uint(__uint_as_float(v[j + q]) * inv);
+                            st_global_v8(dst + (size_t)(o0 + j / 8) * kHeads * 8, o[0], o[1], o[2], o[3], o[4], o[5],
+                                         o[6], o[7]);
+                        }
                     }
                     if (r == 0)
                         args.part_lse[slot * kHeads + m] = l_sum > 0.f ? m_used + __log2f(l_sum) : -CUDART_INF_F;
@@ -733,6 +756,7 @@ __global__ void __launch_bounds__(kAttThreads, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(kBarOFree));
                 if (threadIdx.x == 64) MLA_TRACE_POINT(7, g);
+                if (threadIdx.x == 64) MLA_TRACE_POINT(5, kTraceProlog);
                 m_used = -CUDART_INF_F;
                 l_sum = 0.f;
             }
@@ -746,7 +770,9 @@ __global__ void __launch_bounds__(kAttThreads, 1)
     if (warp == 1) tmem_dealloc(tmem, kTmemCols);
     // The peer may still copy scores into this CTA's shared memory or arrive
     // on its barriers: neither CTA leaves before both are done.
+    if (threadIdx.x == 0) MLA_TRACE_POINT(6, kTraceProlog);
     cluster_sync();
+    if (threadIdx.x == 0) MLA_TRACE_POINT(7, kTraceProlog);
 }
 
 // ------------------------------------------------------------------ plan
@@ -824,113 +850,133 @@ __global__ void __launch_bounds__(32) mla_plan_kernel(const int32_t* __restrict_
 
 // ------------------------------------------------------------------ combine
 
-// Merge of split partials: o_lat = sum_s 2^(lse_s - M) o_s / sum_s 2^(lse_s - M)
-// with M = max_s lse_s (the softmax of the pieces' log-sum-exps).
-//
-// One thread per (split unit, 4 latent columns, head, piece group): the 128
-// consecutive threads of a group read the 128 heads of one column quad, a
-// contiguous 2 KiB of the head-minor partials.  A CTA covers KPC column
-// quads; its G groups take every G-th piece and keep a running (max, sum,
-// accumulator) each, merged through shared memory at the end.  G = 1 suits
-// batches whose sequences are cut into a few pieces; G = 8 gives small
-// batches (a sequence cut into tens of pieces) enough loads in flight.
-// A split unit is (split sequence, query token): blockIdx / per-unit CTAs.
-template <int G, int KPC>
-__global__ void __launch_bounds__(128 * G * KPC) mla_combine_kernel(const Plan* __restrict__ plan,
-                                                                    const float* __restrict__ part_o,
-                                                                    const float* __restrict__ part_lse,
-                                                                    __nv_bfloat16* __restrict__ o_lat) {
-    constexpr int kPerUnit = (kLat / 4) / KPC;  // CTAs per split unit
-    constexpr int kBatch = 4;                   // pieces whose loads are issued together
-    __shared__ float4 s_acc[G > 1 ? G : 1][KPC][kHeads];
-    __shared__ float2 s_mw[G > 1 ? G : 1][KPC][kHeads];
-    pdl_wait();
-    pdl_trigger();
-    const int q_len = plan->q_len;
-    const int work = blockIdx.x / kPerUnit;
-    if (work >= plan->n_split * q_len) return;
-    const int h = threadIdx.x % kHeads;
-    const int kk = (threadIdx.x / kHeads) % KPC;
-    const int g = threadIdx.x / (kHeads * KPC);
-    const int k = (blockIdx.x % kPerUnit) * KPC + kk;  // column quad
-    const int b = plan_splits(plan)[work / q_len];
-    const int qi = work % q_len;
-    const int u = b * q_len + qi;
-    const int* pre = plan_prefix(plan);
-    const int L = plan->L, ovh = plan->ovh;
-    const int tiles = plan_tiles(pre, b, ovh);
-    const int c_lo = pre[b], c_hi = pre[b + 1];
-    const int p_lo = c_lo / L, p_hi = (c_hi - 1) / L;
+// The pieces of query token qi of sequence b: groups p_lo..p_hi, piece p
+// stored in partial slot (p + b) * q_len + qi if its clip of the sequence's
+// tiles is non-empty.  split = false when one group holds the whole
+// sequence (o_lat was then written directly, or zeroed for an invalid
+// length).
+struct UnitPieces {
+    int p_lo, p_hi, c_lo, tiles, L, ovh;
+    bool split;
+    __device__ void init(const Plan* plan, int b) {
+        const int* pre = plan_prefix(plan);
+        L = plan->L;
+        ovh = plan->ovh;
+        c_lo = pre[b];
+        const int c_hi = pre[b + 1];
+        tiles = c_hi > c_lo ? c_hi - c_lo - ovh : 0;
+        p_lo = c_lo / L;
+        p_hi = c_hi > c_lo ? (c_hi - 1) / L : p_lo;
+        split = c_hi > c_lo && (c_lo + ovh) / L != (c_hi - 1) / L;
+    }
     // Group p holds tiles [p L - c_lo - ovh, (p+1) L - c_lo - ovh) of the
     // sequence, clipped to [0, tiles); an empty clip wrote no partial.
-    auto nonempty = [&](int p) {
+    __device__ bool nonempty(int p) const {
         int s0 = p * L - c_lo - ovh, e0 = (p + 1) * L - c_lo - ovh;
         s0 = s0 < 0 ? 0 : (s0 > tiles ? tiles : s0);
         e0 = e0 < 0 ? 0 : (e0 > tiles ? tiles : e0);
         return e0 > s0;
-    };
-    const float4* po = reinterpret_cast<const float4*>(part_o) + (size_t)k * kHeads + h;
-    float m = -CUDART_INF_F, wsum = 0.f;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int p0 = p_lo + g; p0 <= p_hi; p0 += G * kBatch) {
-        float lse[kBatch];
-        float4 v[kBatch];
+    }
+};
+
+// Running merge state of split partials for one (unit, head), lane l
+// holding columns 4(l + 32 j) .. +3, j = 0..3: max m of the pieces' base-2
+// LSEs, sum of 2^(lse - m), and sum of 2^(lse - m) o_p (the softmax of the
+// pieces' log-sum-exps, unnormalised).
+struct MergeState {
+    float m, wsum;
+    float4 acc[4];
+    __device__ void clear() {
+        m = -CUDART_INF_F;
+        wsum = 0.f;
 #pragma unroll
-        for (int j = 0; j < kBatch; ++j) {
-            const int p = p0 + j * G;
-            lse[j] = -CUDART_INF_F;
-            v[j] = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (p <= p_hi && nonempty(p)) {
-                const size_t slot = (size_t)(p + b) * q_len + qi;
-                lse[j] = __ldg(part_lse + slot * kHeads + h);
-                v[j] = __ldg(po + slot * (kLat / 4) * kHeads);
-            }
-        }
-        float mb = m;
+        for (int j = 0; j < 4; ++j) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    // Folds in another state (m2, w2, a2).
+    __device__ void fold(float m2, float w2, const float4 (&a2)[4]) {
+        const float mb = fmaxf(m, m2);
+        if (mb == -CUDART_INF_F) return;
+        const float r0 = exp2f(m - mb), r1 = exp2f(m2 - mb);  // -inf gives 0
+        wsum = wsum * r0 + w2 * r1;
 #pragma unroll
-        for (int j = 0; j < kBatch; ++j) mb = fmaxf(mb, lse[j]);
-        if (mb == -CUDART_INF_F) continue;  // nothing but empty pieces so far
-        const float rr = exp2f(m - mb);     // m = -inf gives 0
-        wsum *= rr;
-        acc.x *= rr;
-        acc.y *= rr;
-        acc.z *= rr;
-        acc.w *= rr;
-#pragma unroll
-        for (int j = 0; j < kBatch; ++j) {
-            const float wgt = exp2f(lse[j] - mb);  // empty piece: 2^-inf = 0
-            wsum += wgt;
-            acc.x += wgt * v[j].x;
-            acc.y += wgt * v[j].y;
-            acc.z += wgt * v[j].z;
-            acc.w += wgt * v[j].w;
+        for (int j = 0; j < 4; ++j) {
+            acc[j].x = acc[j].x * r0 + a2[j].x * r1; acc[j].y = acc[j].y * r0 + a2[j].y * r1;
+            acc[j].z = acc[j].z * r0 + a2[j].z * r1; acc[j].w = acc[j].w * r0 + a2[j].w * r1;
         }
         m = mb;
     }
-    if constexpr (G > 1) {
-        s_acc[g][kk][h] = acc;
-        s_mw[g][kk][h] = make_float2(m, wsum);
-        __syncthreads();
-        if (g != 0) return;
-        for (int j = 1; j < G; ++j) {
-            const float2 mw = s_mw[j][kk][h];
-            const float mb = fmaxf(m, mw.x);
-            if (mb == -CUDART_INF_F) continue;
-            const float r0 = exp2f(m - mb), r1 = exp2f(mw.x - mb);
-            const float4 a1 = s_acc[j][kk][h];
-            wsum = wsum * r0 + mw.y * r1;
-            acc.x = acc.x * r0 + a1.x * r1;
-            acc.y = acc.y * r0 + a1.y * r1;
-            acc.z = acc.z * r0 + a1.z * r1;
-            acc.w = acc.w * r0 + a1.w * r1;
-            m = mb;
+    __device__ void normalise() {
+        const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            acc[j].x *= inv; acc[j].y *= inv; acc[j].z *= inv; acc[j].w *= inv;
         }
     }
-    const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
-    uint2 o;
-    o.x = pack_bf16(acc.x * inv, acc.y * inv);
-    o.y = pack_bf16(acc.z * inv, acc.w * inv);
-    *reinterpret_cast<uint2*>(o_lat + ((size_t)u * kHeads + h) * kLat + 4 * k) = o;
+};
+
+// Adds pieces p_lo + first, p_lo + first + step, ... of one (unit, head) to
+// `st` (one warp); pieces are read four at a time so that their loads
+// overlap.
+__device__ __forceinline__ void merge_pieces_warp(const UnitPieces& up, int b, int qi, int q_len, int h,
+                                                  const float* __restrict__ part_o,
+                                                  const float* __restrict__ part_lse, int lane, int first, int step,
+                                                  MergeState& st) {
+    for (int p0 = up.p_lo + first; p0 <= up.p_hi; p0 += 4 * step) {
+        float lse[4];
+        float4 v[4][4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int p = p0 + i * step;
+            lse[i] = -CUDART_INF_F;
+            if (p <= up.p_hi && up.nonempty(p)) {
+                const size_t slot = (size_t)(p + b) * q_len + qi;
+                lse[i] = __ldg(part_lse + slot * kHeads + h);
+                // columns 4q..4q+3, q = lane + 32 j: octet q / 2, half q % 2
+                const float4* src = reinterpret_cast<const float4*>(part_o) + (slot * (kLat / 8) * kHeads + h) * 2;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int q = lane + 32 * j;
+                    v[i][j] = __ldg(src + (size_t)(q / 2) * kHeads * 2 + (q % 2));
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) v[i][j] = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) st.fold(lse[i], lse[i] == -CUDART_INF_F ? 0.f : 1.f, v[i]);
+    }
+}
+
+// Split combine as its own step: one warp per (split unit, head), eight
+// heads per CTA; writes o_lat (bf16) of the split units.
+__global__ void __launch_bounds__(256) mla_combine_kernel(const Plan* __restrict__ plan,
+                                                          const float* __restrict__ part_o,
+                                                          const float* __restrict__ part_lse,
+                                                          __nv_bfloat16* __restrict__ o_lat) {
+    pdl_wait();
+    pdl_trigger();
+    const int q_len = plan->q_len;
+    const int work = blockIdx.x / (kHeads / 8);
+    if (work >= plan->n_split * q_len) return;
+    const int lane = threadIdx.x % 32;
+    const int h = (blockIdx.x % (kHeads / 8)) * 8 + threadIdx.x / 32;
+    const int b = plan_splits(plan)[work / q_len];
+    const int qi = work % q_len;
+    UnitPieces up;
+    up.init(plan, b);
+    MergeState ms;
+    ms.clear();
+    merge_pieces_warp(up, b, qi, q_len, h, part_o, part_lse, lane, 0, 1, ms);
+    ms.normalise();
+    uint2* dst = reinterpret_cast<uint2*>(o_lat + ((size_t)(b * q_len + qi) * kHeads + h) * kLat) + lane;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        uint2 o;
+        o.x = pack_bf16(ms.acc[j].x, ms.acc[j].y);
+        o.y = pack_bf16(ms.acc[j].z, ms.acc[j].w);
+        dst[32 * j] = o;
+    }
 }
 
 }  // namespace sm100

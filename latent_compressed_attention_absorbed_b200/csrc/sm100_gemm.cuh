@@ -156,6 +156,46 @@ __global__ void __launch_bounds__(128, 1)
         mla_plan_warp(args.seqlens, args.plan_B, args.q_len, args.plan_T_max, args.plan_clusters, args.plan_ovh,
                       args.plan_min_units, args.plan, args.status, args.plan_olat, lane);
     __syncwarp();
+    if (ROPE && warp >= 2) {
+        // q_hat[u][h][512 + 2k..] = RoPE(q_rope[u][h], m_u) for the rows of this
+        // tile, pairs 16y..16y+15 in the CTA with N-tile y, m_u = seqlens[b] -
+        // q_len + i; four pairs (16 bytes) per item, four items' loads in flight
+        // per thread, while the MMAs run.
+        const int tid2 = threadIdx.x - 64;
+        const int items = min(128, args.rows - m0) * 4;
+        for (int it0 = tid2; it0 < items; it0 += 64 * 4) {
+            uint4 x[4];
+            int pos[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int it = it0 + 64 * j;
+                if (it < items) {
+                    const int u = m0 + it / 4, k0 = 16 * blockIdx.y + 4 * (it % 4);
+                    x[j] = __ldg(reinterpret_cast<const uint4*>(args.q_rope + ((size_t)u * args.H + h) * 64 + 2 * k0));
+                    const int b = u / args.q_len, i = u % args.q_len;
+                    pos[j] = args.seqlens[b] - args.q_len + i;
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int it = it0 + 64 * j;
+                if (it < items) {
+                    const int u = m0 + it / 4, k0 = 16 * blockIdx.y + 4 * (it % 4);
+                    const uint32_t in[4] = {x[j].x, x[j].y, x[j].z, x[j].w};
+                    uint32_t o[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        float y0, y1;
+                        mla_rope_rotate(__uint_as_float(in[q] << 16), __uint_as_float(in[q] & 0xffff0000u),
+                                        args.rope.inv_freq[k0 + q], pos[j], &y0, &y1);
+                        o[q] = pack_bf16(y0, y1);
+                    }
+                    *reinterpret_cast<uint4*>(args.out + ((size_t)u * args.H + h) * args.ld_out + 512 + 2 * k0) =
+                        make_uint4(o[0], o[1], o[2], o[3]);
+                }
+            }
+        }
+    }
 
     // ---------------- epilogue: all four warps, TMEM lane quarter = warp
     const bool ok = mbar_wait(done_bar, 0) && !*abort_flag;
@@ -182,21 +222,6 @@ __global__ void __launch_bounds__(128, 1)
         }
     } else if (threadIdx.x == 0) {
         atomicOr(args.status, MLA_STATUS_TIMEOUT);
-    }
-    if (ROPE) {
-        // q_hat[u][h][512 + 2k..] = RoPE(q_rope[u][h], m_u) for the rows of this tile, one pair per item,
-        // pairs 16y..16y+15 in the CTA with N-tile y: m_u = seqlens[b] - q_len + i.
-        const int nrows = min(128, args.rows - m0);
-        for (int item = threadIdx.x; item < nrows * 16; item += blockDim.x) {
-            const int u = m0 + item / 16, k = 16 * blockIdx.y + item % 16;
-            const int b = u / args.q_len, i = u % args.q_len;
-            const int m = args.seqlens[b] - args.q_len + i;
-            const __nv_bfloat162 x = reinterpret_cast<const __nv_bfloat162*>(args.q_rope + ((size_t)u * args.H + h) * 64)[k];
-            float y0, y1;
-            mla_rope_rotate(__low2float(x), __high2float(x), args.rope.inv_freq[k], m, &y0, &y1);
-            reinterpret_cast<__nv_bfloat162*>(args.out + ((size_t)u * args.H + h) * args.ld_out + 512)[k] =
-                __floats2bfloat162_rn(y0, y1);
-        }
     }
     tc_fence_before();
     __syncthreads();

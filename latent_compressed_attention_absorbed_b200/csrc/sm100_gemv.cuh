@@ -1,0 +1,248 @@
+// The two per-head projections of absorbed MLA for small batches (at most
+// eight query tokens), where they are matrix-vector products bound by the
+// weight reads (16.8 MB each):
+//
+//   absorb  (a2): q_lat[u][h][:] = W_UK[h]^T q_nope[u][h][:]   (128 -> 512)
+//                 plus the RoPE of q_R at the query position
+//   project (a5): out[u][h][:]   = W_UV[h] o_lat[u][h][:]      (512 -> 128)
+//
+// (092 page, section 二 "缓存压缩也可以做一个代数检查": fold U^T into the query
+// once; ailearn.mscapital.top MLA panel: W_UV after the latent aggregation.)
+//
+// Each CTA stages its 64 KB slice of the weights in shared memory with
+// cp.async before waiting for the previous kernel (weights are never
+// written by it), so the weight stream overlaps the previous kernel's tail.
+// The project kernel also merges the split-KV partials of the attention
+// step itself (so the decode needs no separate combine launch for these
+// batches).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <math_constants.h>
+
+#include "mla_rope.cuh"
+#include "sm100_attend.cuh"
+#include "sm100_ptx.cuh"
+
+namespace mla {
+namespace sm100 {
+
+constexpr int kGemvMaxRows = 8;
+constexpr int kGemvWBytes = 64 * 1024;  // weight slice of one CTA
+template <int R> constexpr int absorb_gemv_smem() { return kGemvWBytes + R * 128 * 4; }
+constexpr int kMergeStateFloats = kLat + 4;  // acc[512], m, wsum (padded)
+constexpr int kProjWarps = 16;                // project CTA: 512 threads, all 128 output rows of a head
+constexpr int kProjWBytes = 128 * kLat * 2;   // W_UV[h]: 128 KB
+template <int R> constexpr int project_gemv_smem() { return kProjWBytes + R * kLat * 4 + kProjWarps * kMergeStateFloats * 4; }
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+__device__ __forceinline__ float2 bf16x2_to_f2(uint32_t v) {
+    return make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u));
+}
+
+struct AbsorbGemvArgs {
+    const __nv_bfloat16* q_nope;  // [rows][128][128]
+    const __nv_bfloat16* q_rope;  // [rows][128][64]
+    const __nv_bfloat16* W_UK;    // [128][128][512]
+    const int32_t* seqlens;       // [B]
+    int rows, q_len;
+    __nv_bfloat16* q_hat;         // [rows][128][576]
+    RopeTable rope;
+    int* status;
+    // split plan of the attention step, written by CTA (128, 0)
+    Plan* plan;
+    int plan_B, plan_T_max, plan_clusters, plan_ovh, plan_min_units;
+    __nv_bfloat16* plan_olat;
+};
+
+// grid (129, 2), 128 threads: CTA (h, y) produces latent columns
+// 256y..256y+255 of head h for every row and RoPE pairs 16y..16y+15; CTA
+// (128, 0) writes the attention plan.  Thread t owns columns 2t, 2t+1.
+template <int R>
+__global__ void __launch_bounds__(128) absorb_gemv_kernel(AbsorbGemvArgs a) {
+    extern __shared__ __align__(16) uint8_t gemv_smem[];
+    auto w_s = reinterpret_cast<__nv_bfloat16(*)[256]>(gemv_smem);                 // W_UK[h][d][256y ..]
+    auto q_s = reinterpret_cast<float(*)[128]>(gemv_smem + kGemvWBytes);          // q_nope rows, fp32
+    const int h = blockIdx.x, y = blockIdx.y, t = threadIdx.x;
+    if (h == kHeads) {
+        pdl_wait();
+        if (y == 0 && t < 32 && a.plan)
+            mla_plan_warp(a.seqlens, a.plan_B, a.q_len, a.plan_T_max, a.plan_clusters, a.plan_ovh,
+                          a.plan_min_units, a.plan, a.status, a.plan_olat, t);
+        if (t == 0) pdl_trigger();
+        return;
+    }
+    // weights first (they do not depend on the previous kernel): 128 rows x 512 B
+    {
+        const uint32_t ws = smem_u32(&w_s[0][0]);
+        const __nv_bfloat16* src = a.W_UK + (size_t)h * 128 * kLat + 256 * y;
+#pragma unroll 4
+        for (int i = t; i < 128 * 32; i += 128) {
+            const int d = i / 32, c = i % 32;
+            cp_async16(ws + d * 512 + c * 16, src + (size_t)d * kLat + c * 8);
+        }
+    }
+    pdl_wait();
+    if (t == 0) pdl_trigger();
+    for (int i = t; i < R * 128; i += 128) {
+        const int u = i / 128, d = i % 128;
+        q_s[u][d] = u < a.rows ? __bfloat162float(a.q_nope[((size_t)u * kHeads + h) * 128 + d]) : 0.f;
+    }
+    // RoPE of q_R at the query position m = T_b - q_len + i (pairs 16y..16y+15)
+    if (t < R * 16) {
+        const int u = t / 16, k = 16 * y + t % 16;
+        if (u < a.rows) {
+            const int b = u / a.q_len, i = u % a.q_len;
+            const int m = a.seqlens[b] - a.q_len + i;
+            const __nv_bfloat162 x =
+                reinterpret_cast<const __nv_bfloat162*>(a.q_rope + ((size_t)u * kHeads + h) * kRope)[k];
+            float y0, y1;
+            mla_rope_rotate(__low2float(x), __high2float(x), a.rope.inv_freq[k], m, &y0, &y1);
+            reinterpret_cast<__nv_bfloat162*>(a.q_hat + ((size_t)u * kHeads + h) * kRow + kLat)[k] =
+                __floats2bfloat162_rn(y0, y1);
+        }
+    }
+    cp_async_wait_all();
+    __syncthreads();
+    float acc[R][2];
+#pragma unroll
+    for (int u = 0; u < R; ++u) acc[u][0] = acc[u][1] = 0.f;
+    const uint32_t* wrow = reinterpret_cast<const uint32_t*>(&w_s[0][0]) + t;
+#pragma unroll 8
+    for (int d = 0; d < 128; ++d) {
+        const float2 w = bf16x2_to_f2(wrow[d * 128]);
+#pragma unroll
+        for (int u = 0; u < R; ++u) {
+            const float q = q_s[u][d];
+            acc[u][0] = fmaf(w.x, q, acc[u][0]);
+            acc[u][1] = fmaf(w.y, q, acc[u][1]);
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < R; ++u)
+        if (u < a.rows)
+            reinterpret_cast<__nv_bfloat162*>(a.q_hat + ((size_t)u * kHeads + h) * kRow + 256 * y)[t] =
+                __floats2bfloat162_rn(acc[u][0], acc[u][1]);
+}
+
+struct ProjectGemvArgs {
+    const Plan* plan;             // split plan (decode path)
+    const __nv_bfloat16* o_lat;   // [rows][128][512]: unsplit units (and zeroed invalid ones)
+    const float* part_o;          // [slots][128][512]
+    const float* part_lse;        // [slots][128]
+    const __nv_bfloat16* W_UV;    // [128][128][512]
+    int rows;
+    __nv_bfloat16* out;           // [rows][128][128]
+};
+
+// grid (128), 512 threads: CTA h produces all 128 output columns of head h.
+// With R rows and G = 16 / R warps per row, warp w serves row u = w % R as
+// member g = w / R of its group:
+//   1. o_lat of row u in fp32: read directly (unit not split), or merged from
+//      the split partials, each warp of the group taking every G-th piece and
+//      the group's states combined through shared memory;
+//   2. output rows v = g * 8R .. + 8R - 1 of row u: dot(W_UV[h][v], o),
+//      lane l covering latent columns 16l..16l+15.
+template <int R>
+__global__ void __launch_bounds__(512) project_gemv_kernel(ProjectGemvArgs a) {
+    constexpr int G = kProjWarps / R;
+    extern __shared__ __align__(16) uint8_t gemv_smem[];
+    auto w_s = reinterpret_cast<__nv_bfloat16(*)[kLat]>(gemv_smem);                    // W_UV[h][v][:]
+    auto o_s = reinterpret_cast<float(*)[kLat]>(gemv_smem + kProjWBytes);              // o_lat rows, fp32
+    auto st_s = reinterpret_cast<float(*)[kMergeStateFloats]>(gemv_smem + kProjWBytes + R * kLat * 4);
+    const int h = blockIdx.x, t = threadIdx.x;
+    const int warp = t / 32, lane = t % 32;
+    const int u = warp % R, g = warp / R;
+    {
+        const uint32_t ws = smem_u32(&w_s[0][0]);
+        const __nv_bfloat16* src = a.W_UV + (size_t)h * 128 * kLat;
+#pragma unroll 4
+        for (int i = t; i < kProjWBytes / 16; i += 512) cp_async16(ws + i * 16, src + (size_t)i * 8);
+    }
+    pdl_wait();
+    if (t == 0) pdl_trigger();
+    // ---- 1. o_lat of row u
+    bool split = false;
+    UnitPieces up;
+    int b = 0, qi = 0, q_len = 1;
+    if (u < a.rows && a.plan) {
+        q_len = a.plan->q_len;
+        b = u / q_len;
+        qi = u % q_len;
+        up.init(a.plan, b);
+        split = up.split;
+    }
+    if (split) {
+        MergeState ms;
+        ms.clear();
+        merge_pieces_warp(up, b, qi, q_len, h, a.part_o, a.part_lse, lane, g, G, ms);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) reinterpret_cast<float4*>(&st_s[warp][0])[lane + 32 * j] = ms.acc[j];
+        if (lane == 0) {
+            st_s[warp][kLat] = ms.m;
+            st_s[warp][kLat + 1] = ms.wsum;
+        }
+    } else if (g == 0) {
+        const uint2* src = reinterpret_cast<const uint2*>(a.o_lat + ((size_t)u * kHeads + h) * kLat) + lane;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint2 v = u < a.rows ? src[32 * j] : make_uint2(0, 0);
+            const float2 lo = bf16x2_to_f2(v.x), hi = bf16x2_to_f2(v.y);
+            reinterpret_cast<float4*>(&o_s[u][0])[lane + 32 * j] = make_float4(lo.x, lo.y, hi.x, hi.y);
+        }
+    }
+    __syncthreads();
+    if (split && g == 0) {
+        MergeState ms;
+        ms.clear();
+        for (int k = 0; k < G; ++k) {
+            const int wk = u + R * k;
+            float4 a2[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) a2[j] = reinterpret_cast<const float4*>(&st_s[wk][0])[lane + 32 * j];
+            ms.fold(st_s[wk][kLat], st_s[wk][kLat + 1], a2);
+        }
+        ms.normalise();
+        // the merged value is what the unsplit path holds: bf16 o_lat
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float2 lo = bf16x2_to_f2(pack_bf16(ms.acc[j].x, ms.acc[j].y));
+            const float2 hi = bf16x2_to_f2(pack_bf16(ms.acc[j].z, ms.acc[j].w));
+            reinterpret_cast<float4*>(&o_s[u][0])[lane + 32 * j] = make_float4(lo.x, lo.y, hi.x, hi.y);
+        }
+    }
+    cp_async_wait_all();
+    __syncthreads();
+    // ---- 2. output rows of row u handled by this warp
+    float o[16];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const float4 v = reinterpret_cast<const float4*>(&o_s[u][16 * lane])[j];
+        o[4 * j] = v.x; o[4 * j + 1] = v.y; o[4 * j + 2] = v.z; o[4 * j + 3] = v.w;
+    }
+#pragma unroll 2
+    for (int vv = 0; vv < 8 * R; ++vv) {
+        const int v = g * 8 * R + vv;
+        const uint4* wr = reinterpret_cast<const uint4*>(&w_s[v][16 * lane]);
+        const uint4 w0 = wr[0], w1 = wr[1];
+        const uint32_t ww[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+        float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float2 w = bf16x2_to_f2(ww[j]);
+            s0 = fmaf(w.x, o[2 * j], s0);
+            s1 = fmaf(w.y, o[2 * j + 1], s1);
+        }
+        float sum = s0 + s1;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+        if (lane == 0 && u < a.rows) a.out[((size_t)u * kHeads + h) * 128 + v] = __float2bfloat16_rn(sum);
+    }
+}
+
+}  // namespace sm100
+}  // namespace mla
