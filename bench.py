@@ -420,13 +420,18 @@ def main():
     kern, step_work = work(cfg)
     bw = pk["hbm_gbs"] * 1e9
     fl = pk["bf16_tflops"] * 1e12
-    # dominant kernel: largest share of the step
+    # dominant kernel: largest share of the step.  Kernel names follow the
+    # library's dispatch: matrix-vector absorb up to 2 query rows and
+    # matrix-vector project (with the split merge) up to 8 rows, tensor-core
+    # GEMMs (and a separate combine kernel) above.
+    rows = cfg.B * cfg.q_len
     dom = max(("absorb", "attend", "project"), key=lambda k: stage_ms[k])
     kt = stage_ms[dom] * 1e-3
     kb, kf = kern[dom]["bytes"], kern[dom]["flops"]
     hbm_bound = kb / bw >= kf / fl
-    kname = {"absorb": "head_gemm_kernel (W_UK absorb)", "attend": "mla_attend_kernel",
-             "project": "head_gemm_kernel (W_UV project)"}[dom]
+    kname = {"absorb": "absorb_gemv_kernel" if rows <= 2 else "head_gemm_kernel (W_UK absorb)",
+             "attend": "mla_attend_kernel",
+             "project": "project_gemv_kernel" if rows <= 8 else "head_gemm_kernel (W_UV project)"}[dom]
     traffic = traffic_for(cfg.name, kname)
     roof = {"kernel": kname, "bound": "hbm" if hbm_bound else "tensor",
             "achieved": round((kb / kt / 1e9) if hbm_bound else (kf / kt / 1e12), 2),
@@ -462,7 +467,8 @@ def main():
         "step_roofline_frac": round(step_roof_s / t_step, 4),
         "stage_us": {k: round(v * 1e3, 3) for k, v in stage_ms.items()},
         "roofline": roof,
-        "gpu_launches": (6 if path == "sm100" else 4) * args.steps * args.gpus,
+        # append + absorb + attend (+ combine above 8 query rows) + project per step
+        "gpu_launches": ((4 if rows <= 8 else 5) if path == "sm100" else 4) * args.steps * args.gpus,
         "clocks": clocks,
         "e2e": e2e,
     }
