@@ -354,10 +354,16 @@ int mla_decode_ex(const mla_dims_t* dims, const void* q_nope, const void* q_rope
         e = B * q_len <= kSmallAbsorbRows ? sm100_absorb_small(p, q_nope, q_rope, W_UK, seqlens, q_hat, st, &pr)
                                           : sm100_absorb(p, q_nope, q_rope, W_UK, seqlens, q_hat, st, &pr);
         ev.record(MLA_EV_ABSORB_DONE, st);
+        // When the cache read is small the HBM idles during attention: prefetch
+        // W_UV into L2 meanwhile (the cache bound is a cheap host-side bound:
+        // B sequences of at most T_max rows).
+        const size_t cache_bound = (size_t)B * cv.T_max * (p.d_c + p.d_r) * 2;
+        const bool pf = cache_bound <= (size_t(64) << 20);
         if (e == cudaSuccess)
             e = sm100_attend(p, q_hat, cv, seqlens, o_lat, ws + L.attend, L.total - L.attend, pairs,
                              opts ? opts->overhead_tiles : -1, opts ? opts->min_tiles : 0, status, st, &ev,
-                             /*plan_ready=*/true, /*combine=*/!small);
+                             /*plan_ready=*/true, /*combine=*/!small, pf ? W_UV : nullptr,
+                             (size_t)p.H * p.d_v * p.d_c * 2);
         ev.record(MLA_EV_COMBINE_DONE, st);
         if (e == cudaSuccess)
             e = small ? sm100_project_small(p, ws + L.attend, pairs, o_lat, W_UV, out, st)

@@ -85,7 +85,8 @@ cudaError_t sm100_absorb(const Problem& p, const void* q_nope, const void* q_rop
 cudaError_t sm100_attend(const Problem& p, const void* q_hat, const CacheView& cache, const int32_t* seqlens,
                          void* o_lat, void* workspace, size_t ws_bytes, int num_pairs, int overhead_tiles,
                          int min_tiles, int* status, cudaStream_t st, const Events* events = nullptr,
-                         bool plan_ready = false, bool combine = true);
+                         bool plan_ready = false, bool combine = true, const void* prefetch = nullptr,
+                         size_t prefetch_bytes = 0);
 cudaError_t sm100_project(const Problem& p, const void* o_lat, const void* W_UV, int rows, void* out,
                           cudaStream_t st);
 // Small batches: matrix-vector kernels.  The project step (B * q_len <= 8)

@@ -324,7 +324,7 @@ size_t sm100_attend_workspace_bytes(const Problem& p, int num_pairs) {
 cudaError_t sm100_attend(const Problem& p, const void* q_hat, const CacheView& cache, const int32_t* seqlens,
                          void* o_lat, void* workspace, size_t ws_bytes, int num_pairs, int overhead_tiles,
                          int min_tiles, int* status, cudaStream_t st, const Events* events, bool plan_ready,
-                         bool combine) {
+                         bool combine, const void* prefetch, size_t prefetch_bytes) {
     const int clusters = attend_clusters(num_pairs, p.q_len);
     size_t off_part, off_lse;
     const size_t need = attend_layout(p, clusters, &off_part, &off_lse);
@@ -361,6 +361,8 @@ cudaError_t sm100_attend(const Problem& p, const void* q_hat, const CacheView& c
     a.q_hat = (const __nv_bfloat16*)q_hat;
     a.o_lat = (__nv_bfloat16*)o_lat;
     a.o_lat_v8 = (reinterpret_cast<uintptr_t>(o_lat) & 31u) == 0;
+    a.prefetch = static_cast<const uint8_t*>(prefetch);
+    a.prefetch_bytes = prefetch ? prefetch_bytes : 0;
     a.part_o = reinterpret_cast<float*>(ws + off_part);
     a.part_lse = reinterpret_cast<float*>(ws + off_lse);
     a.status = status;

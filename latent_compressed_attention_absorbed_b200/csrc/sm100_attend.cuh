@@ -32,10 +32,10 @@
 // groups writes fp32 partials plus a base-2 LSE per head and token, merged by
 // the combine kernel.
 //
-// Roles per CTA (320 threads):
+// Roles per CTA (352 threads):
 //   warp 0     TMA producer (stage ring, L2 prefetch of the tiles ahead);
-//   warp 1     TMEM owner and MMA issuer (event loop: O as soon as P is
-//              published, S as soon as its tile and the S buffer are free);
+//   warp 1     TMEM owner and issuer of the score MMAs (S);
+//   warp 10    issuer of the P.V MMAs (O), as soon as P is published;
 //   warps 2-5  softmax: add the two partial scores, online softmax, P into
 //              TMEM, rescale / normalise O, write o_lat or split partials;
 //   warps 6-9  exchange: read partial S out of TMEM, publish it (local copy
@@ -95,7 +95,7 @@ constexpr int kTmemO = 0;     // O: 256 fp32 latent columns of this CTA's half
 constexpr int kTmemS = 256;   // S: 64 fp32 partial scores
 constexpr int kTmemP = 320;   // P: two buffers of 64 bf16 probabilities, two per column
 constexpr int kTmemQ = 384;   // Q-hat latent half: 256 bf16, two per column (128 columns)
-constexpr int kAttThreads = 320;
+constexpr int kAttThreads = 352;
 
 // Barrier indices (8 bytes each) inside the barrier block.
 enum {
@@ -234,6 +234,8 @@ struct AttendArgs {
     const __nv_bfloat16* q_hat;   // [B][q_len][128][576]
     __nv_bfloat16* o_lat;         // [B][q_len][128][512]
     int o_lat_v8;                 // o_lat is 32-byte aligned: 32-byte stores
+    const uint8_t* prefetch;      // optional: range prefetched into L2 while the kernel runs
+    size_t prefetch_bytes;        // (the next step's weights when this step's own traffic is small)
     float* part_o;                // [slots][64 column octets][128 heads][8]
     float* part_lse;              // [slots][128]
     int* status;
@@ -309,6 +311,17 @@ __global__ void __launch_bounds__(kAttThreads, 1)
     if (threadIdx.x == 0) pdl_trigger();
     if (threadIdx.x == 0) MLA_TRACE_POINT(2, kTraceProlog);
     const bool active = grp < args.plan->groups;
+    // Warp 0, lanes 1..31: spread the optional L2 prefetch over the grid, 16 KB a request.
+    if (warp == 0 && lane > 0 && args.prefetch) {
+        const size_t per_cta = ((args.prefetch_bytes / gridDim.x) + 16383) & ~size_t(16383);
+        const size_t lo = per_cta * blockIdx.x;
+        for (size_t off = lo + 16384 * (size_t)(lane - 1); off < lo + per_cta && off < args.prefetch_bytes;
+             off += 16384 * 31) {
+            const size_t n = args.prefetch_bytes - off < 16384 ? args.prefetch_bytes - off : 16384;
+            prefetch_l2_bulk(args.prefetch + off, (uint32_t)(n & ~size_t(15)));
+        }
+    }
+
     const int quarter = warp & 3;
     const int m = quarter * 32 + lane;                          // head / TMEM lane (warps 2..9)
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;  // the warp's TMEM subpartition
@@ -349,71 +362,30 @@ __global__ void __launch_bounds__(kAttThreads, 1)
             }
         }
     } else if (warp == 1) {
-        // ======================================================== MMA issuer (whole warp polls, lane 0 issues)
+        // ======================================================== S issuer (whole warp waits, lane 0 issues)
         constexpr uint32_t idS = idesc_bf16_f32(kHeads, kNk, false, false);
-        constexpr uint32_t idO = idesc_bf16_f32(kHeads, kHalfLat, false, true);
         const uint32_t stages = base + kOffStages;
         // Descriptor templates: the start-address field (bits 0..13, address >> 4)
         // is advanced by adding byte offsets >> 4.
         const uint64_t dLatK = smem_desc(stages, 16, 1024, kSw128);       // cache latent, K-major (S)
         const uint64_t dRopeK = smem_desc(stages, 16, 512, kSw64);        // cache RoPE, K-major (S)
-        const uint64_t dLatMN = smem_desc(stages, kChunk, 1024, kSw128);  // cache latent, MN-major (O)
         const uint64_t dQR = smem_desc(base + kOffQR, 16, 512, kSw64);    // Q-hat RoPE half (S, A operand)
-        TileWalk ws, wo;  // next tile whose S / O is issued
+        // S(g) = Q-hat half . cache half^T over this CTA's 288 columns, in tile
+        // order: each S waits for its piece's Q-hat, its tile and S(g-1) to be
+        // read out of TMEM.  (The O MMAs are issued by warp 10: issuing blocks
+        // at the tensor pipe's pace, and a ready O must not wait behind an S.)
+        TileWalk ws;
         ws.init(args.plan, grp);
-        wo = ws;
-        int gs = 0, go = 0;
-        int T_s = ws.valid ? args.seqlens[ws.seq] : 0;  // length of the sequence of tile gs
-        // Warp-uniform non-blocking barrier probe (lane 0 decides).
-        auto ready = [&](uint32_t b, uint32_t parity) -> bool {
-            return __shfl_sync(0xffffffffu, mbar_test_wait(b, parity) ? 1 : 0, 0) != 0;
-        };
-        // O += P(g) . cache latent half(g); the first tile of a piece overwrites
-        // O (after the previous piece's epilogue has read it).
-        auto o_ready = [&]() -> bool {
-            if (!wo.valid || !ready(bar(kBarPFull0 + (go & 1)), (go >> 1) & 1)) return false;
-            return !(wo.first() && wo.seg > 0) || ready(bar(kBarOFree), (wo.seg - 1) & 1);
-        };
-        auto issue_O = [&]() {
-            const int g = go;
-            const bool first = wo.first(), last = wo.last();
-            tc_fence_after();
-            if (lane == 0) {
-                MLA_TRACE_POINT(15, g);
-                const int st = g % kStages;
-                const uint64_t dB = dLatMN + ((kOffStages + st * kStageBytes) >> 4);
-                const uint32_t pA = tmem + kTmemP + 32 * (g & 1);
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    mma_f16_ts(tmem + kTmemO, pA + 8 * k, dB + ((2048 * k) >> 4), idO, (!first || k > 0) ? 1u : 0u);
-                mma_commit(bar(kBarPFree0 + (g & 1)));
-                mma_commit(bar(kBarEmpty0 + st));
-                if (last) mma_commit(bar(kBarOFull));
-                MLA_TRACE_POINT(2, g);
-            }
-            __syncwarp();
-            ++go;
-            wo.advance();
-        };
-        // S(g) = Q-hat half . cache half^T over this CTA's 288 columns: it needs
-        // the piece's Q-hat, the tile, and S(g-1) read out of TMEM.
-        auto s_ready = [&]() -> bool {
-            const int g = gs;
-            if (!ws.valid) return false;
-            if (ws.first() && !ready(bar(kBarQFull), ws.seg & 1)) return false;
-            if (!ready(bar(kBarFull0 + g % kStages), (g / kStages) & 1)) return false;
-#ifdef MLA_TRACE
-            if (lane == 0 && g < kTraceTiles && g_mla_trace[r][g][10] == 0 && cl == MLA_TRACE_CLUSTER)
-                MLA_TRACE_POINT(10, g);
-#endif
-            return g == 0 || ready(bar(kBarSFree), (g - 1) & 1);
-        };
-        // The 18 MMAs of S go out in three groups; a pending O is issued between
-        // groups (issuing runs at the tensor pipe's pace), so O(g) never waits
-        // for a whole S.
-        auto issue_S = [&]() {
-            const int g = gs;
+        int T_s = ws.valid ? args.seqlens[ws.seq] : 0;  // length of the sequence of tile g
+        bool ok = true;
+        for (int g = 0; ws.valid && ok && !*abort_flag; ++g) {
+            if (ws.first() && !mbar_wait(bar(kBarQFull), ws.seg & 1)) { ok = false; break; }
             const uint32_t tile_off = kOffStages + (g % kStages) * kStageBytes;
+            if (!mbar_wait(bar(kBarFull0 + g % kStages), (g / kStages) & 1)) { ok = false; break; }
+#ifdef MLA_TRACE
+            if (lane == 0) MLA_TRACE_POINT(10, g);
+#endif
+            if (g > 0 && !mbar_wait(bar(kBarSFree), (g - 1) & 1)) { ok = false; break; }
             const int valid = T_s - ws.t * kNk;
             if (valid < kNk) {
                 // Rows at or beyond T_b hold no cached token: zero the latent
@@ -426,59 +398,60 @@ __global__ void __launch_bounds__(kAttThreads, 1)
             }
             __syncwarp();
             tc_fence_after();
-            const uint32_t dS = tmem + kTmemS;
-            const uint64_t dL = dLatK + (tile_off >> 4);
-            if (lane == 0) MLA_TRACE_POINT(14, g);
+            if (lane == 0) {
+                MLA_TRACE_POINT(14, g);
+#ifdef MLA_TRACE_CYCLES
+                const long long c_s0 = clock64();
+#endif
+                const uint32_t dS = tmem + kTmemS;
+                const uint64_t dL = dLatK + (tile_off >> 4);
 #pragma unroll
-            for (int grp6 = 0; grp6 < 3; ++grp6) {
-                if (lane == 0) {
+                for (int k = 0; k < 16; ++k)
+                    mma_f16_ts(dS, tmem + kTmemQ + 8 * k, dL + (((k >> 2) * kChunk + 32 * (k & 3)) >> 4), idS,
+                               k ? 1u : 0u);
 #pragma unroll
-                    for (int kk = 0; kk < 6; ++kk) {
-                        const int k = 6 * grp6 + kk;
-                        if (k < 16) {
-                            mma_f16_ts(dS, tmem + kTmemQ + 8 * k, dL + (((k >> 2) * kChunk + 32 * (k & 3)) >> 4),
-                                       idS, k ? 1u : 0u);
-                        } else {
-                            const int j = k - 16;
-                            mma_f16_ss(dS, dQR + ((32 * j) >> 4), dRopeK + ((tile_off + 4 * kChunk + 32 * j) >> 4),
-                                       idS, 1u);
-                        }
-                    }
-                    if (grp6 == 2) {
-                        mma_commit(bar(kBarSFull));
-                        MLA_TRACE_POINT(1, g);
-                    }
-                }
-                __syncwarp();
-                if (grp6 < 2 && o_ready()) issue_O();
+                for (int j = 0; j < 2; ++j)
+                    mma_f16_ss(dS, dQR + ((32 * j) >> 4), dRopeK + ((tile_off + 4 * kChunk + 32 * j) >> 4), idS, 1u);
+                mma_commit(bar(kBarSFull));
+                MLA_TRACE_POINT(1, g);
+#ifdef MLA_TRACE_CYCLES
+                if (cl == MLA_TRACE_CLUSTER && g < kTraceTiles) g_mla_trace[r][g][11] = (unsigned long long)(clock64() - c_s0);
+#endif
             }
-            ++gs;
+            __syncwarp();
             const int seq_before = ws.seq;
             ws.advance();
             if (ws.valid && ws.seq != seq_before) T_s = args.seqlens[ws.seq];
-        };
-        // Event loop: O first (it frees a stage and a P buffer), then S.  Every
-        // dependency of an S or O points to earlier tiles, so polling both
-        // cannot deadlock.
+        }
+        if (!ok) *abort_flag = 1;
+    } else if (warp == 10) {
+        // ======================================================== O issuer (whole warp waits, lane 0 issues)
+        // O += P(g) . cache latent half(g); the first tile of a piece overwrites
+        // O (after the previous piece's epilogue has read it).
+        constexpr uint32_t idO = idesc_bf16_f32(kHeads, kHalfLat, false, true);
+        const uint64_t dLatMN = smem_desc(base + kOffStages, kChunk, 1024, kSw128);  // cache latent, MN-major
+        TileWalk wo;
+        wo.init(args.plan, grp);
         bool ok = true;
-        uint64_t t_idle = 0;
-        while (wo.valid && !*abort_flag) {
-            bool progress = false;
-            if (o_ready()) {
-                issue_O();
-                progress = true;
-            } else if (s_ready()) {
-                issue_S();
-                progress = true;
+        for (int g = 0; wo.valid && ok && !*abort_flag; ++g, wo.advance()) {
+            if (!mbar_wait(bar(kBarPFull0 + (g & 1)), (g >> 1) & 1)) { ok = false; break; }
+            if (wo.first() && wo.seg > 0 && !mbar_wait(bar(kBarOFree), (wo.seg - 1) & 1)) { ok = false; break; }
+            tc_fence_after();
+            if (lane == 0) {
+                MLA_TRACE_POINT(15, g);
+                const bool first = wo.first();
+                const int st = g % kStages;
+                const uint64_t dB = dLatMN + ((kOffStages + st * kStageBytes) >> 4);
+                const uint32_t pA = tmem + kTmemP + 32 * (g & 1);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    mma_f16_ts(tmem + kTmemO, pA + 8 * k, dB + ((2048 * k) >> 4), idO, (!first || k > 0) ? 1u : 0u);
+                mma_commit(bar(kBarPFree0 + (g & 1)));
+                mma_commit(bar(kBarEmpty0 + st));
+                if (wo.last()) mma_commit(bar(kBarOFull));
+                MLA_TRACE_POINT(2, g);
             }
-            if (progress) {
-                t_idle = 0;
-            } else if (t_idle == 0) {
-                t_idle = global_timer_ns();
-            } else if (global_timer_ns() - t_idle > MLA_WAIT_LIMIT_NS) {
-                ok = false;
-                break;
-            }
+            __syncwarp();
         }
         if (!ok) *abort_flag = 1;
     } else if (warp >= 6) {
@@ -696,8 +669,10 @@ __global__ void __launch_bounds__(kAttThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(kBarPFull0 + b2));
             if (threadIdx.x == 64) MLA_TRACE_POINT(6, g);
+#ifndef MLA_TRACE_CYCLES
             if (threadIdx.x == 96) MLA_TRACE_POINT(11, g);
             if (threadIdx.x == 128) MLA_TRACE_POINT(12, g);
+#endif
             if (threadIdx.x == 160) MLA_TRACE_POINT(13, g);
             // ---- epilogue at the end of a piece: this thread owns O row m (256 columns)
             if (w.last()) {
