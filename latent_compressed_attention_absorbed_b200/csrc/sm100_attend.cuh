@@ -85,7 +85,8 @@ constexpr int kOffOwn = kOffStages + kStages * kStageBytes;
 constexpr int kOffX = kOffOwn + 2 * kXBytes;
 constexpr int kQRBytes = kHeads * 64;                  // 8192
 constexpr int kOffQR = kOffX + 2 * kXBytes;
-constexpr int kOffBars = kOffQR + kQRBytes;
+constexpr int kOffRed = kOffQR + kQRBytes;            // softmax pair exchange: [2][2][128] fp32
+constexpr int kOffBars = kOffRed + 2 * 2 * kHeads * 4;
 constexpr int kAttSmem = kOffBars + 256 + 1024;
 static_assert(kAttSmem <= 232448, "attention kernel shared memory exceeds 227 KB");
 
@@ -95,7 +96,7 @@ constexpr int kTmemO = 0;     // O: 256 fp32 latent columns of this CTA's half
 constexpr int kTmemS = 256;   // S: 64 fp32 partial scores
 constexpr int kTmemP = 320;   // P: two buffers of 64 bf16 probabilities, two per column
 constexpr int kTmemQ = 384;   // Q-hat latent half: 256 bf16, two per column (128 columns)
-constexpr int kAttThreads = 352;
+constexpr int kAttThreads = 512;
 
 // Barrier indices (8 bytes each) inside the barrier block.
 enum {
@@ -279,15 +280,15 @@ __global__ void __launch_bounds__(kAttThreads, 1)
         mbar_init(bar(kBarSFull), 1);
         mbar_init(bar(kBarSFree), 4);
         for (int s = 0; s < 2; ++s) {
-            mbar_init(bar(kBarPFull0 + s), 4);
+            mbar_init(bar(kBarPFull0 + s), 8);
             mbar_init(bar(kBarPFree0 + s), 1);
             mbar_init(bar(kBarOwnFull0 + s), 4);
-            mbar_init(bar(kBarOwnFree0 + s), 4);
+            mbar_init(bar(kBarOwnFree0 + s), 8);
             mbar_init(bar(kBarXFull0 + s), 1);
-            mbar_init(bar(kBarXFree0 + s), 4);
+            mbar_init(bar(kBarXFree0 + s), 8);
         }
         mbar_init(bar(kBarOFull), 1);
-        mbar_init(bar(kBarOFree), 4);
+        mbar_init(bar(kBarOFree), 8);
         *abort_flag = 0;
         fence_mbar_init();
         prefetch_tensormap(&mapLat);
@@ -454,7 +455,9 @@ __global__ void __launch_bounds__(kAttThreads, 1)
             __syncwarp();
         }
         if (!ok) *abort_flag = 1;
-    } else if (warp >= 6) {
+    } else if (warp == 11) {
+        // spare warp (keeps the softmax halves on the same SMSPs as their quarters)
+    } else if (warp >= 6 && warp <= 9) {
         // ======================================================== exchange warps 6..9
         const float sl2 = args.scale_log2;
         const uint32_t x_peer = mapa(base + kOffX, peer);
@@ -501,10 +504,16 @@ __global__ void __launch_bounds__(kAttThreads, 1)
             tc_fence_after();
             uint32_t own[32];
             {
-                uint32_t va[32], vb[32];
-                tmem_ld32(tmem + lane_addr + kTmemS, va);
-                tmem_ld32(tmem + lane_addr + kTmemS + 32, vb);
-                tmem_wait_ld();
+                // two 32-column halves, each packed as soon as it arrives
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    uint32_t va[32];
+                    tmem_ld32(tmem + lane_addr + kTmemS + 32 * hf, va);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        own[16 * hf + j] = pack_f16(__uint_as_float(va[2 * j]) * sl2, __uint_as_float(va[2 * j + 1]) * sl2);
+                }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(kBarSFree));
@@ -514,11 +523,6 @@ __global__ void __launch_bounds__(kAttThreads, 1)
                     TileWalk nx = w;
                     nx.advance();
                     if (nx.valid) load_q(nx.seq * q_len + qi);
-                }
-#pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    own[j] = pack_f16(__uint_as_float(va[2 * j]) * sl2, __uint_as_float(va[2 * j + 1]) * sl2);
-                    own[16 + j] = pack_f16(__uint_as_float(vb[2 * j]) * sl2, __uint_as_float(vb[2 * j + 1]) * sl2);
                 }
             }
             // ---- publish: Own[hb] (read by our softmax warps and by the bulk copy
@@ -562,30 +566,30 @@ __global__ void __launch_bounds__(kAttThreads, 1)
         }
         if (!ok) *abort_flag = 1;
     } else {
-        // ======================================================== softmax warps 2..5
+        // ======================================================== softmax warps 2..5 and 12..15
+        // Two warps per TMEM quarter: half kh takes keys 32kh..32kh+31 of each
+        // score row and latent columns 128kh..128kh+127 of O; the pair agrees on
+        // the row maximum through shared memory (named barrier 1 + quarter).
+        const int kh = warp >= 12 ? 1 : 0;
         const uint32_t xfree_peer = mapa(bar(kBarXFree0), peer);
+        float* red = reinterpret_cast<float*>(base_ptr + kOffRed);  // [2 tiles][2 halves][128 rows]
         bool ok = true;
         TileWalk w;
         w.init(args.plan, grp);
-        float m_used = -CUDART_INF_F, l_sum = 0.f;
+        float m_used = -CUDART_INF_F, l_part = 0.f;
         int n_keys = 0;
         for (int g = 0; w.valid && ok && !*abort_flag; ++g, w.advance()) {
             const int b2 = g & 1;
-            // ---- S(g) = own partial + the peer's, added in the same order on both CTAs
+            // ---- S(g) for this thread's 32 keys = own partial + the peer's (same order on both CTAs)
             if (!mbar_wait(bar(kBarOwnFull0 + b2), (g >> 1) & 1)) { ok = false; break; }
-#ifndef MLA_NO_XCHG
             if (!mbar_wait_cluster(bar(kBarXFull0 + b2), (g >> 1) & 1)) { ok = false; break; }
-#endif
-            float s[kNk];
+            float s[32];
             {
                 const uint32_t own_buf = base + kOffOwn + b2 * kXBytes;
-#ifdef MLA_NO_XCHG
-                const uint32_t x_buf = own_buf;
-#else
                 const uint32_t x_buf = base + kOffX + b2 * kXBytes;
-#endif
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
+                for (int cc = 0; cc < 4; ++cc) {
+                    const int c = 4 * kh + cc;
                     uint32_t a0, a1, a2, a3, o0, o1, o2, o3;
                     ld_shared_v4u(own_buf + sw128(m, c), a0, a1, a2, a3);
                     ld_shared_v4u(x_buf + sw128(m, c), o0, o1, o2, o3);
@@ -594,8 +598,8 @@ __global__ void __launch_bounds__(kAttThreads, 1)
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         const float2 v = sum_f16x2(mine[q], oth[q]);
-                        s[8 * c + 2 * q] = v.x;
-                        s[8 * c + 2 * q + 1] = v.y;
+                        s[8 * cc + 2 * q] = v.x;
+                        s[8 * cc + 2 * q + 1] = v.y;
                     }
                 }
             }
@@ -604,36 +608,37 @@ __global__ void __launch_bounds__(kAttThreads, 1)
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive(bar(kBarOwnFree0 + b2));
-#ifndef MLA_NO_XCHG
                 mbar_arrive_remote_relaxed(xfree_peer + 8 * b2);
-#endif
             }
             if (threadIdx.x == 64) MLA_TRACE_POINT(5, g);
             // ---- online softmax in base 2, lazy rescaling of O
             // query token qi of sequence b sees keys 0..T_b-q_len+qi
             if (w.first()) n_keys = args.seqlens[w.seq] - q_len + 1 + qi;
-            const int key0 = w.t * kNk;
-            if (key0 + kNk > n_keys) {
+            const int key0 = w.t * kNk + 32 * kh;
+            if (key0 + 32 > n_keys) {
 #pragma unroll
-                for (int j = 0; j < kNk; ++j)
+                for (int j = 0; j < 32; ++j)
                     if (key0 + j >= n_keys) s[j] = -CUDART_INF_F;
             }
             float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
 #pragma unroll
-            for (int j = 4; j < kNk; j += 4) {
+            for (int j = 4; j < 32; j += 4) {
                 mx0 = fmaxf(mx0, s[j]); mx1 = fmaxf(mx1, s[j + 1]);
                 mx2 = fmaxf(mx2, s[j + 2]); mx3 = fmaxf(mx3, s[j + 3]);
             }
-            const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+            float* rg = red + (b2 * 2) * kHeads;  // this tile's [2 halves][128 rows]
+            rg[kh * kHeads + m] = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+            named_bar_sync(1 + quarter, 64);
+            const float mx = fmaxf(rg[m], rg[kHeads + m]);
             if (threadIdx.x == 64) MLA_TRACE_POINT(8, g);
             const bool first = w.first();
             const bool grow = mx > m_used + 8.0f;  // rescale only when the max grows by > 2^8
             const float mb_new = grow ? mx : m_used;
             const float mb = (mb_new == -CUDART_INF_F) ? 0.f : mb_new;
-            uint32_t pk[32];
+            uint32_t pk[16];
             float rs0 = 0.f, rs1 = 0.f;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
+            for (int j = 0; j < 16; ++j) {
                 const float p0 = ex2(s[2 * j] - mb), p1 = ex2(s[2 * j + 1] - mb);
                 rs0 += p0;
                 rs1 += p1;
@@ -648,22 +653,22 @@ __global__ void __launch_bounds__(kAttThreads, 1)
                     if (!mbar_wait(bar(kBarPFree0 + (b2 ^ 1)), ((g - 1) >> 1) & 1)) { ok = false; break; }
                     tc_fence_after();
                     const float f = ex2(m_used - mx);
-                    l_sum *= f;
+                    l_part *= f;
 #pragma unroll 1
-                    for (int c0 = 0; c0 < kHalfLat; c0 += 32) {
+                    for (int c0 = 0; c0 < kHalfLat / 2; c0 += 32) {
                         uint32_t v[32];
-                        tmem_ld32(tmem + lane_addr + kTmemO + c0, v);
+                        tmem_ld32(tmem + lane_addr + kTmemO + 128 * kh + c0, v);
                         tmem_wait_ld();
 #pragma unroll
                         for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * f);
-                        tmem_st32(tmem + lane_addr + kTmemO + c0, v);
+                        tmem_st32(tmem + lane_addr + kTmemO + 128 * kh + c0, v);
                     }
                 }
                 m_used = mx;
             }
             tc_fence_after();
-            l_sum += rs0 + rs1;
-            tmem_st32(tmem + lane_addr + kTmemP + 32 * b2, pk);
+            l_part += rs0 + rs1;
+            tmem_st16(tmem + lane_addr + kTmemP + 32 * b2 + 16 * kh, pk);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
@@ -671,22 +676,28 @@ __global__ void __launch_bounds__(kAttThreads, 1)
             if (threadIdx.x == 64) MLA_TRACE_POINT(6, g);
 #ifndef MLA_TRACE_CYCLES
             if (threadIdx.x == 96) MLA_TRACE_POINT(11, g);
-            if (threadIdx.x == 128) MLA_TRACE_POINT(12, g);
+            if (threadIdx.x == 384) MLA_TRACE_POINT(12, g);
 #endif
             if (threadIdx.x == 160) MLA_TRACE_POINT(13, g);
-            // ---- epilogue at the end of a piece: this thread owns O row m (256 columns)
+            // ---- epilogue at the end of a piece: this thread owns O row m, columns 128kh..+127
             if (w.last()) {
+                // the row's softmax denominator: both halves' partial sums
+                float* rl = red + (b2 * 2) * kHeads;
+                named_bar_sync(1 + quarter, 64);  // the pair has read this tile's maxima
+                rl[kh * kHeads + m] = l_part;
+                named_bar_sync(1 + quarter, 64);
+                const float l_sum = rl[m] + rl[kHeads + m];
                 if (!mbar_wait(bar(kBarOFull), w.seg & 1)) { ok = false; break; }
                 tc_fence_after();
-                if (threadIdx.x == 64) MLA_TRACE_POINT(4, kTraceProlog);
                 const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
                 const int u = w.seq * q_len + qi;
+                const int col0 = r * kHalfLat + 128 * kh;  // first latent column of this thread
                 if (w.whole) {
-                    __nv_bfloat16* dst = args.o_lat + ((size_t)u * kHeads + m) * kLat + r * kHalfLat;
+                    __nv_bfloat16* dst = args.o_lat + ((size_t)u * kHeads + m) * kLat + col0;
 #pragma unroll 1
-                    for (int c0 = 0; c0 < kHalfLat; c0 += 32) {
+                    for (int c0 = 0; c0 < kHalfLat / 2; c0 += 32) {
                         uint32_t v[32];
-                        tmem_ld32(tmem + lane_addr + kTmemO + c0, v);
+                        tmem_ld32(tmem + lane_addr + kTmemO + 128 * kh + c0, v);
                         tmem_wait_ld();
 #pragma unroll
                         for (int j = 0; j < 32; j += 16) {
@@ -710,11 +721,11 @@ __global__ void __launch_bounds__(kAttThreads, 1)
                     const size_t slot = (size_t)(grp + w.seq) * q_len + qi;
                     float* dst = args.part_o + (slot * (kLat / 8) * kHeads + m) * 8;
 #pragma unroll 1
-                    for (int c0 = 0; c0 < kHalfLat; c0 += 32) {
+                    for (int c0 = 0; c0 < kHalfLat / 2; c0 += 32) {
                         uint32_t v[32];
-                        tmem_ld32(tmem + lane_addr + kTmemO + c0, v);
+                        tmem_ld32(tmem + lane_addr + kTmemO + 128 * kh + c0, v);
                         tmem_wait_ld();
-                        const int o0 = (r * kHalfLat + c0) / 8;
+                        const int o0 = (col0 + c0) / 8;
 #pragma unroll
                         for (int j = 0; j < 32; j += 8) {
                             uint32_t o[8];
@@ -724,7 +735,7 @@ __global__ void __launch_bounds__(kAttThreads, 1)
                                          o[6], o[7]);
                         }
                     }
-                    if (r == 0)
+                    if (r == 0 && kh == 0)
                         args.part_lse[slot * kHeads + m] = l_sum > 0.f ? m_used + __log2f(l_sum) : -CUDART_INF_F;
                 }
                 tc_fence_before();
@@ -733,7 +744,7 @@ __global__ void __launch_bounds__(kAttThreads, 1)
                 if (threadIdx.x == 64) MLA_TRACE_POINT(7, g);
                 if (threadIdx.x == 64) MLA_TRACE_POINT(5, kTraceProlog);
                 m_used = -CUDART_INF_F;
-                l_sum = 0.f;
+                l_part = 0.f;
             }
         }
         if (!ok) *abort_flag = 1;
