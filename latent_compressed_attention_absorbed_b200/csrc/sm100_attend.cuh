@@ -504,19 +504,19 @@ __global__ void __launch_bounds__(kAttThreads, 1)
             tc_fence_after();
             uint32_t own[32];
             {
-                // two 32-column halves, each packed as soon as it arrives
-#pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
-                    uint32_t va[32];
-                    tmem_ld32(tmem + lane_addr + kTmemS + 32 * hf, va);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int j = 0; j < 16; ++j)
-                        own[16 * hf + j] = pack_f16(__uint_as_float(va[2 * j]) * sl2, __uint_as_float(va[2 * j + 1]) * sl2);
-                }
+                // both halves out of TMEM first, so that S(h+1) may start at once
+                uint32_t va[32], vb[32];
+                tmem_ld32(tmem + lane_addr + kTmemS, va);
+                tmem_ld32(tmem + lane_addr + kTmemS + 32, vb);
+                tmem_wait_ld();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(kBarSFree));
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    own[j] = pack_f16(__uint_as_float(va[2 * j]) * sl2, __uint_as_float(va[2 * j + 1]) * sl2);
+                    own[16 + j] = pack_f16(__uint_as_float(vb[2 * j]) * sl2, __uint_as_float(vb[2 * j + 1]) * sl2);
+                }
                 if (threadIdx.x == 192) MLA_TRACE_POINT(3, h);
                 // S(h) was the last reader of this piece's Q-hat: load the next piece's.
                 if (w.last()) {
