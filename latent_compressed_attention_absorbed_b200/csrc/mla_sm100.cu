@@ -197,6 +197,7 @@ cudaError_t sm100_absorb(const Problem& p, const void* q_nope, const void* q_rop
     a.ld_out = kRow;
     a.out_col0 = 0;
     a.out = (__nv_bfloat16*)q_hat;
+    a.out_v8 = (reinterpret_cast<uintptr_t>(q_hat) & 31u) == 0;
     a.q_rope = (const __nv_bfloat16*)q_rope;
     a.seqlens = seqlens;
     a.q_len = p.q_len;
@@ -240,6 +241,7 @@ cudaError_t sm100_project(const Problem& p, const void* o_lat, const void* W_UV,
     a.ld_out = 128;
     a.out_col0 = 0;
     a.out = (__nv_bfloat16*)out;
+    a.out_v8 = (reinterpret_cast<uintptr_t>(out) & 31u) == 0;
     a.status = device_status_ptr();
     a.q_len = 1;
     a.a_rows = gemm_a_rows(rows);

@@ -36,6 +36,7 @@ struct GemmArgs {
     int q_len;
     RopeTable rope;
     int a_rows;       // rows of each A box (multiple of 16, <= 128)
+    int out_v8;       // out is 32-byte aligned: 32-byte stores in the epilogue
     int* status;
     // split plan of the attention step, written by warp 2 of CTA (0,0,0) when non-null
     Plan* plan;
@@ -210,13 +211,16 @@ __global__ void __launch_bounds__(128, 1)
             if (row < args.rows) {
                 __nv_bfloat16* dst = args.out + ((size_t)row * args.H + h) * args.ld_out + args.out_col0 + n0 + c0;
 #pragma unroll
-                for (int j = 0; j < 32; j += 8) {
-                    uint4 v;
-                    v.x = pack_bf16(__uint_as_float(r[j + 0]), __uint_as_float(r[j + 1]));
-                    v.y = pack_bf16(__uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]));
-                    v.z = pack_bf16(__uint_as_float(r[j + 4]), __uint_as_float(r[j + 5]));
-                    v.w = pack_bf16(__uint_as_float(r[j + 6]), __uint_as_float(r[j + 7]));
-                    *reinterpret_cast<uint4*>(dst + j) = v;
+                for (int j = 0; j < 32; j += 16) {
+                    uint32_t o[8];
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) o[q] = pack_bf16(__uint_as_float(r[j + 2 * q]), __uint_as_float(r[j + 2 * q + 1]));
+                    if (args.out_v8) {
+                        st_global_v8(dst + j, o[0], o[1], o[2], o[3], o[4], o[5], o[6], o[7]);
+                    } else {
+                        *reinterpret_cast<uint4*>(dst + j) = make_uint4(o[0], o[1], o[2], o[3]);
+                        *reinterpret_cast<uint4*>(dst + j + 8) = make_uint4(o[4], o[5], o[6], o[7]);
+                    }
                 }
             }
         }

@@ -31,9 +31,12 @@ constexpr int kGemvMaxRows = 8;
 constexpr int kGemvWBytes = 64 * 1024;  // weight slice of one CTA
 template <int R> constexpr int absorb_gemv_smem() { return kGemvWBytes + R * 128 * 4; }
 constexpr int kMergeStateFloats = kLat + 4;  // acc[512], m, wsum (padded)
-constexpr int kProjWarps = 16;                // project CTA: 512 threads, all 128 output rows of a head
-constexpr int kProjWBytes = 128 * kLat * 2;   // W_UV[h]: 128 KB
-template <int R> constexpr int project_gemv_smem() { return kProjWBytes + R * kLat * 4 + kProjWarps * kMergeStateFloats * 4; }
+constexpr int kProjWarps = 16;                 // project CTA: 512 threads, all 128 output rows of a head
+constexpr int kProjWRow = kLat * 2 + 16;       // W_UV row in shared memory, padded: lanes hit distinct banks
+constexpr int kProjWBytes = 128 * kProjWRow;   // W_UV[h]: 130 KB
+template <int R> constexpr int project_gemv_smem() {
+    return kProjWBytes + R * kLat * 4 + kProjWarps * kMergeStateFloats * 4 + 4 * R * 128 * 4;
+}
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
@@ -145,23 +148,29 @@ struct ProjectGemvArgs {
 //   1. o_lat of row u in fp32: read directly (unit not split), or merged from
 //      the split partials, each warp of the group taking every G-th piece and
 //      the group's states combined through shared memory;
-//   2. output rows v = g * 8R .. + 8R - 1 of row u: dot(W_UV[h][v], o),
-//      lane l covering latent columns 16l..16l+15.
+//   2. thread (v, q) forms the dot products of output row v with every row
+//      over latent columns 128q..128q+127; the four partial sums are added
+//      through shared memory.
 template <int R>
 __global__ void __launch_bounds__(512) project_gemv_kernel(ProjectGemvArgs a) {
     constexpr int G = kProjWarps / R;
     extern __shared__ __align__(16) uint8_t gemv_smem[];
-    auto w_s = reinterpret_cast<__nv_bfloat16(*)[kLat]>(gemv_smem);                    // W_UV[h][v][:]
+    uint8_t* w_s = gemv_smem;                                                          // W_UV[h][v][:], padded rows
     auto o_s = reinterpret_cast<float(*)[kLat]>(gemv_smem + kProjWBytes);              // o_lat rows, fp32
     auto st_s = reinterpret_cast<float(*)[kMergeStateFloats]>(gemv_smem + kProjWBytes + R * kLat * 4);
+    auto sum_s = reinterpret_cast<float(*)[R][128]>(gemv_smem + kProjWBytes + R * kLat * 4 +
+                                                     kProjWarps * kMergeStateFloats * 4);  // [4 column quarters][R][v]
     const int h = blockIdx.x, t = threadIdx.x;
     const int warp = t / 32, lane = t % 32;
     const int u = warp % R, g = warp / R;
     {
-        const uint32_t ws = smem_u32(&w_s[0][0]);
+        const uint32_t ws = smem_u32(w_s);
         const __nv_bfloat16* src = a.W_UV + (size_t)h * 128 * kLat;
 #pragma unroll 4
-        for (int i = t; i < kProjWBytes / 16; i += 512) cp_async16(ws + i * 16, src + (size_t)i * 8);
+        for (int i = t; i < 128 * 64; i += 512) {
+            const int v = i / 64, c = i % 64;  // row v, 16-byte chunk c
+            cp_async16(ws + v * kProjWRow + c * 16, src + (size_t)v * kLat + c * 8);
+        }
     }
     pdl_wait();
     if (t == 0) pdl_trigger();
@@ -217,30 +226,41 @@ __global__ void __launch_bounds__(512) project_gemv_kernel(ProjectGemvArgs a) {
     }
     cp_async_wait_all();
     __syncthreads();
-    // ---- 2. output rows of row u handled by this warp
-    float o[16];
+    // ---- 2. out[u][h][v] = sum_c W_UV[h][v][c] o[u][c]: thread (v, quarter q) takes
+    // output row v = t % 128 and latent columns 128q..128q+127 for every row u;
+    // the four quarters are added through shared memory.
+    {
+        const int v = t % 128, q = t / 128;
+        float acc[R];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const float4 v = reinterpret_cast<const float4*>(&o_s[u][16 * lane])[j];
-        o[4 * j] = v.x; o[4 * j + 1] = v.y; o[4 * j + 2] = v.z; o[4 * j + 3] = v.w;
-    }
+        for (int uu = 0; uu < R; ++uu) acc[uu] = 0.f;
+        const uint8_t* wrow = w_s + v * kProjWRow + q * 256;
 #pragma unroll 2
-    for (int vv = 0; vv < 8 * R; ++vv) {
-        const int v = g * 8 * R + vv;
-        const uint4* wr = reinterpret_cast<const uint4*>(&w_s[v][16 * lane]);
-        const uint4 w0 = wr[0], w1 = wr[1];
-        const uint32_t ww[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-        float s0 = 0.f, s1 = 0.f;
+        for (int c8 = 0; c8 < 16; ++c8) {
+            const uint4 w8 = *reinterpret_cast<const uint4*>(wrow + c8 * 16);
+            const float2 w01 = bf16x2_to_f2(w8.x), w23 = bf16x2_to_f2(w8.y);
+            const float2 w45 = bf16x2_to_f2(w8.z), w67 = bf16x2_to_f2(w8.w);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const float2 w = bf16x2_to_f2(ww[j]);
-            s0 = fmaf(w.x, o[2 * j], s0);
-            s1 = fmaf(w.y, o[2 * j + 1], s1);
+            for (int uu = 0; uu < R; ++uu) {
+                const float4 o0 = *reinterpret_cast<const float4*>(&o_s[uu][128 * q + 8 * c8]);
+                const float4 o1 = *reinterpret_cast<const float4*>(&o_s[uu][128 * q + 8 * c8 + 4]);
+                float x = acc[uu];
+                x = fmaf(w01.x, o0.x, x); x = fmaf(w01.y, o0.y, x);
+                x = fmaf(w23.x, o0.z, x); x = fmaf(w23.y, o0.w, x);
+                x = fmaf(w45.x, o1.x, x); x = fmaf(w45.y, o1.y, x);
+                x = fmaf(w67.x, o1.z, x); x = fmaf(w67.y, o1.w, x);
+                acc[uu] = x;
+            }
         }
-        float sum = s0 + s1;
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-        if (lane == 0 && u < a.rows) a.out[((size_t)u * kHeads + h) * 128 + v] = __float2bfloat16_rn(sum);
+        for (int uu = 0; uu < R; ++uu) sum_s[q][uu][v] = acc[uu];
+    }
+    __syncthreads();
+    for (int i = t; i < R * 128; i += 512) {
+        const int uu = i / 128, v = i % 128;
+        if (uu < a.rows)
+            a.out[((size_t)uu * kHeads + h) * 128 + v] =
+                __float2bfloat16_rn(sum_s[0][uu][v] + sum_s[1][uu][v] + sum_s[2][uu][v] + sum_s[3][uu][v]);
     }
 }
 
