@@ -20,10 +20,15 @@
 extern "C" int mla_trace_read(void* host, size_t bytes) {
     return cudaMemcpyFromSymbol(host, mla::sm100::g_mla_trace, bytes) == cudaSuccess ? 0 : -4;
 }
+extern "C" int mla_trace_read_all(void* host, size_t bytes) {
+    return cudaMemcpyFromSymbol(host, mla::sm100::g_mla_trace_all, bytes) == cudaSuccess ? 0 : -4;
+}
 extern "C" int mla_trace_clear(void) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, mla::sm100::g_mla_trace) != cudaSuccess) return -4;
-    return cudaMemset(p, 0, sizeof(mla::sm100::g_mla_trace)) == cudaSuccess ? 0 : -4;
+    if (cudaMemset(p, 0, sizeof(mla::sm100::g_mla_trace)) != cudaSuccess) return -4;
+    if (cudaGetSymbolAddress(&p, mla::sm100::g_mla_trace_all) != cudaSuccess) return -4;
+    return cudaMemset(p, 0, sizeof(mla::sm100::g_mla_trace_all)) == cudaSuccess ? 0 : -4;
 }
 #endif
 
@@ -307,7 +312,7 @@ static size_t attend_layout(const Problem& p, int pairs, size_t* off_part, size_
     const int clusters = attend_clusters(pairs, p.q_len);
     Carve c(nullptr);
     const size_t units = (size_t)p.B * p.q_len;  // one per query token
-    c.take(sizeof(Plan) + sizeof(int) * (2 * units + 1));
+    c.take(sizeof(Plan) + sizeof(int) * (kPlanMaxGroups + 2 * units + 1));
     const size_t slots = (size_t)clusters + units;
     *off_part = c.off;
     c.take(slots * kHeads * kLat * sizeof(float));
@@ -328,6 +333,7 @@ cudaError_t sm100_attend(const Problem& p, const void* q_hat, const CacheView& c
                          int min_tiles, int* status, cudaStream_t st, const Events* events, bool plan_ready,
                          bool combine, const void* prefetch, size_t prefetch_bytes) {
     const int clusters = attend_clusters(num_pairs, p.q_len);
+    if (clusters / p.q_len > kPlanMaxGroups) return cudaErrorInvalidValue;
     size_t off_part, off_lse;
     const size_t need = attend_layout(p, clusters, &off_part, &off_lse);
     if (ws_bytes < need) return cudaErrorInvalidValue;

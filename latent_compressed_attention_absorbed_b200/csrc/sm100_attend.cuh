@@ -135,7 +135,19 @@ __device__ unsigned long long g_mla_trace[2][kTraceTiles][16];
     do {                                                                                                  \
         if (cl == MLA_TRACE_CLUSTER && (n) < kTraceTiles) g_mla_trace[r][(n)][(ev)] = global_timer_ns(); \
     } while (0)
+// Per-CTA summary of every cluster: [cluster][rank][8] = entry, after the
+// grid dependency wait, first S issued, last O issued, last epilogue done,
+// exit, tiles, pieces.
+constexpr int kTraceAllClusters = 256;
+__device__ unsigned long long g_mla_trace_all[kTraceAllClusters][2][8];
+#define MLA_TRACE_ALL(ev, value)                                         \
+    do {                                                                 \
+        if (cl < kTraceAllClusters) g_mla_trace_all[cl][r][(ev)] = (value); \
+    } while (0)
 #else
+#define MLA_TRACE_ALL(ev, value) \
+    do {                         \
+    } while (0)
 #define MLA_TRACE_POINT(ev, n) \
     do {                       \
     } while (0)
@@ -154,10 +166,16 @@ struct Plan {
     int q_len;
     int groups;   // groups of q_len clusters
     int pad;
-    // followed by int cost_prefix[B + 1], then int split_seq[B]
+    // followed by int group_first[kPlanMaxGroups] (the sequence holding cost
+    // unit g L, or B past the end), int cost_prefix[B + 1], int split_seq[B]
 };
+// The per-group table sits at a fixed offset, so that a cluster finds its
+// first piece without a search over the prefix sums: the header, the table
+// entry and then two prefix sums are two dependent reads from global memory.
+constexpr int kPlanMaxGroups = 1024;  // the cluster count is capped at 1024
 
-__device__ __forceinline__ const int* plan_prefix(const Plan* p) { return reinterpret_cast<const int*>(p + 1); }
+__device__ __forceinline__ const int* plan_group_first(const Plan* p) { return reinterpret_cast<const int*>(p + 1); }
+__device__ __forceinline__ const int* plan_prefix(const Plan* p) { return plan_group_first(p) + kPlanMaxGroups; }
 __device__ __forceinline__ const int* plan_splits(const Plan* p) { return plan_prefix(p) + p->B + 1; }
 
 // Tiles of sequence b (0 if its length was invalid).
@@ -177,13 +195,7 @@ struct SegIter {
         ovh = plan->ovh;
         lo = grp * L;
         hi = lo + L;
-        // largest b with pre[b] <= lo
-        int a = 0, z = B;
-        while (a < z) {
-            const int mid = (a + z + 1) / 2;
-            if (pre[mid] <= lo) a = mid; else z = mid - 1;
-        }
-        b = a;
+        b = plan_group_first(plan)[grp];  // the sequence whose cost range holds lo
     }
     // Advances to the next non-empty piece; false when done.
     __device__ bool next(int& seq, int& k0, int& k1, bool& whole) {
@@ -271,6 +283,7 @@ __global__ void __launch_bounds__(kAttThreads, 1)
     const int grp = cl / q_len, qi = cl % q_len;
 
     if (threadIdx.x == 0) MLA_TRACE_POINT(0, kTraceProlog);
+    if (threadIdx.x == 0) MLA_TRACE_ALL(0, global_timer_ns());
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(bar(kBarFull0 + s), 1);
@@ -311,6 +324,7 @@ __global__ void __launch_bounds__(kAttThreads, 1)
     pdl_wait();
     if (threadIdx.x == 0) pdl_trigger();
     if (threadIdx.x == 0) MLA_TRACE_POINT(2, kTraceProlog);
+    if (threadIdx.x == 0) MLA_TRACE_ALL(1, global_timer_ns());
     const bool active = grp < args.plan->groups;
     // Warp 0, lanes 1..31: spread the optional L2 prefetch over the grid, 16 KB a request.
     if (warp == 0 && lane > 0 && args.prefetch) {
@@ -332,7 +346,9 @@ __global__ void __launch_bounds__(kAttThreads, 1)
     } else if (warp == 0) {
         // ======================================================== TMA producer (runs up to kStages tiles ahead)
         // Tiles kPrefetch ahead of the loads are prefetched into L2, so that a
-        // stage, once freed, refills at L2 rather than HBM latency.
+        // stage, once freed, refills at L2 rather than HBM latency.  (Issuing the
+        // first loads ahead of the first prefetches measured slower: the early
+        // burst of prefetches keeps HBM busy while the pipeline fills.)
         if (lane == 0) {
             TileWalk w, wp;
             w.init(args.plan, grp);
@@ -344,6 +360,16 @@ __global__ void __launch_bounds__(kAttThreads, 1)
             }
             for (int n = 0; w.valid && !*abort_flag; ++n, w.advance()) {
                 if (kPrefetch > 0 && wp.valid) {
+                    // A later piece's Q-hat (147 KB, contiguous) goes into L2 as the
+                    // look-ahead enters it, ahead of its reload: each CTA of the
+                    // pair prefetches one half, 8 KB a request.
+                    if (wp.first() && wp.seg > 0) {
+                        constexpr uint32_t kQBytes = kHeads * kRow * 2, kPiece = 8192;
+                        const uint8_t* q = reinterpret_cast<const uint8_t*>(args.q_hat) +
+                                           (size_t)(wp.seq * q_len + qi) * kQBytes;
+                        for (uint32_t off = r * (kQBytes / 2); off < (r + 1) * (kQBytes / 2); off += kPiece)
+                            prefetch_l2_bulk(q + off, kPiece);
+                    }
                     tma_prefetch_3d(&mapPf, kHalfLat * r, wp.t * kNk, wp.seq);
                     tma_prefetch_3d(&mapRope, kLat + kHalfRope * r, wp.t * kNk, wp.seq);
                     wp.advance();
@@ -415,6 +441,7 @@ __global__ void __launch_bounds__(kAttThreads, 1)
                     mma_f16_ss(dS, dQR + ((32 * j) >> 4), dRopeK + ((tile_off + 4 * kChunk + 32 * j) >> 4), idS, 1u);
                 mma_commit(bar(kBarSFull));
                 MLA_TRACE_POINT(1, g);
+                if (g == 0) MLA_TRACE_ALL(2, global_timer_ns());
 #ifdef MLA_TRACE_CYCLES
                 if (cl == MLA_TRACE_CLUSTER && g < kTraceTiles) g_mla_trace[r][g][11] = (unsigned long long)(clock64() - c_s0);
 #endif
@@ -451,6 +478,9 @@ __global__ void __launch_bounds__(kAttThreads, 1)
                 mma_commit(bar(kBarEmpty0 + st));
                 if (wo.last()) mma_commit(bar(kBarOFull));
                 MLA_TRACE_POINT(2, g);
+                MLA_TRACE_ALL(3, global_timer_ns());
+                MLA_TRACE_ALL(6, (unsigned long long)(g + 1));
+                MLA_TRACE_ALL(7, (unsigned long long)(wo.seg + 1));
             }
             __syncwarp();
         }
@@ -518,36 +548,17 @@ __global__ void __launch_bounds__(kAttThreads, 1)
                     own[16 + j] = pack_f16(__uint_as_float(vb[2 * j]) * sl2, __uint_as_float(vb[2 * j + 1]) * sl2);
                 }
                 if (threadIdx.x == 192) MLA_TRACE_POINT(3, h);
-                // S(h) was the last reader of this piece's Q-hat: load the next piece's.
-                if (w.last()) {
-                    TileWalk nx = w;
-                    nx.advance();
-                    if (nx.valid) load_q(nx.seq * q_len + qi);
-                }
             }
             // ---- publish: Own[hb] (read by our softmax warps and by the bulk copy
             // into the peer's X[hb]); both readers of tile h-2 must be done.
             if (h >= 2) {
                 if (!mbar_wait(bar(kBarOwnFree0 + hb), ((h >> 1) - 1) & 1)) { ok = false; break; }
-#ifndef MLA_NO_XCHG
                 if (!mbar_wait_cluster(bar(kBarXFree0 + hb), ((h >> 1) - 1) & 1)) { ok = false; break; }
-#endif
             }
             const uint32_t own_buf = base + kOffOwn + hb * kXBytes;
 #pragma unroll
             for (int c = 0; c < 8; ++c)
                 st_shared_v4(own_buf + sw128(m, c), own[4 * c], own[4 * c + 1], own[4 * c + 2], own[4 * c + 3]);
-#ifdef MLA_XCHG_STASYNC
-#pragma unroll
-            for (int c = 0; c < 8; ++c)
-                st_async_v4_b32(x_peer + hb * kXBytes + sw128(m, c), own[4 * c], own[4 * c + 1], own[4 * c + 2],
-                                own[4 * c + 3], xfull_peer + 8 * hb);
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(kBarOwnFull0 + hb));
-#elif defined(MLA_NO_XCHG)
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(kBarOwnFull0 + hb));
-#else
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
@@ -555,13 +566,18 @@ __global__ void __launch_bounds__(kAttThreads, 1)
                 bulk_copy_s2s(x_peer + hb * kXBytes + off, own_buf + off, 32 * 128, xfull_peer + 8 * hb);
                 mbar_arrive(bar(kBarOwnFull0 + hb));
             }
-#endif
             // The peer's partial for tile h lands in our X[hb] (its phase h/2).
             if (threadIdx.x == 192) {
-#ifndef MLA_NO_XCHG
                 mbar_arrive_expect_tx(bar(kBarXFull0 + hb), kXBytes);
-#endif
                 MLA_TRACE_POINT(4, h);
+            }
+            // S(h) was the last reader of this piece's Q-hat: load the next
+            // piece's, after the partial is on its way (the next S waits for it,
+            // the exchange of tile h does not).
+            if (w.last()) {
+                TileWalk nx = w;
+                nx.advance();
+                if (nx.valid) load_q(nx.seq * q_len + qi);
             }
         }
         if (!ok) *abort_flag = 1;
@@ -743,6 +759,7 @@ __global__ void __launch_bounds__(kAttThreads, 1)
                 if (lane == 0) mbar_arrive(bar(kBarOFree));
                 if (threadIdx.x == 64) MLA_TRACE_POINT(7, g);
                 if (threadIdx.x == 64) MLA_TRACE_POINT(5, kTraceProlog);
+                if (threadIdx.x == 64) MLA_TRACE_ALL(4, global_timer_ns());
                 m_used = -CUDART_INF_F;
                 l_part = 0.f;
             }
@@ -759,6 +776,7 @@ __global__ void __launch_bounds__(kAttThreads, 1)
     if (threadIdx.x == 0) MLA_TRACE_POINT(6, kTraceProlog);
     cluster_sync();
     if (threadIdx.x == 0) MLA_TRACE_POINT(7, kTraceProlog);
+    if (threadIdx.x == 0) MLA_TRACE_ALL(5, global_timer_ns());
 }
 
 // ------------------------------------------------------------------ plan
@@ -771,9 +789,11 @@ __global__ void __launch_bounds__(kAttThreads, 1)
 __device__ __forceinline__ void mla_plan_warp(const int32_t* __restrict__ seqlens, int B, int q_len, int T_max,
                                               int clusters, int ovh, int min_units, Plan* plan, int* status,
                                               __nv_bfloat16* o_lat, int lane) {
-    int* pre = reinterpret_cast<int*>(plan + 1);
+    int* gfirst = reinterpret_cast<int*>(plan + 1);
+    int* pre = gfirst + kPlanMaxGroups;
     int* splits = pre + B + 1;
     const int groups = clusters / q_len > 0 ? clusters / q_len : 1;
+    for (int g = lane; g < groups; g += 32) gfirst[g] = B;
     int carry = 0;
     if (lane == 0) pre[0] = 0;
     for (int base = 0; base < B; base += 32) {
@@ -805,6 +825,9 @@ __device__ __forceinline__ void mla_plan_warp(const int32_t* __restrict__ seqlen
             const int lo = pre[b], hi = pre[b + 1];
             if (hi == lo) invalid = true;
             else split = (lo + ovh) / L != (hi - 1) / L;
+            // groups whose first cost unit g L falls in [lo, hi) start in sequence b
+            if (hi > lo)
+                for (int g = (lo + L - 1) / L; g <= (hi - 1) / L && g < groups; ++g) gfirst[g] = b;
         }
         const unsigned msk = __ballot_sync(0xffffffffu, split);
         if (split) splits[n_split + __popc(msk & ((1u << lane) - 1))] = b;

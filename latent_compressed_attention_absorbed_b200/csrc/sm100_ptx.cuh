@@ -144,27 +144,6 @@ __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-// 16-byte store into another CTA's shared memory that completes `bytes` of
-// transaction count on that CTA's mbarrier.
-__device__ __forceinline__ void st_async_v4(uint32_t cluster_addr, float a, float b, float c, float d,
-                                            uint32_t cluster_bar) {
-    asm volatile(
-        "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
-            cluster_addr),
-        "f"(a), "f"(b), "f"(c), "f"(d), "r"(cluster_bar)
-        : "memory");
-}
-
-// Same with four 32-bit words (e.g. eight packed fp16 values).
-__device__ __forceinline__ void st_async_v4_b32(uint32_t cluster_addr, uint32_t a, uint32_t b, uint32_t c,
-                                                uint32_t d, uint32_t cluster_bar) {
-    asm volatile(
-        "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
-            cluster_addr),
-        "r"(a), "r"(b), "r"(c), "r"(d), "r"(cluster_bar)
-        : "memory");
-}
-
 // Bulk copy from this CTA's shared memory to another CTA's (addresses from
 // mapa), completing `bytes` of transaction count on that CTA's mbarrier.
 // Addresses 16-byte aligned, bytes a multiple of 16.
