@@ -49,6 +49,8 @@
 #include <cuda_bf16.h>
 #include <math_constants.h>
 
+#include <climits>
+
 #include "mla_rope.cuh"
 #include "sm100_ptx.cuh"
 
@@ -135,11 +137,34 @@ __device__ unsigned long long g_mla_trace[2][kTraceTiles][16];
     do {                                                                                                  \
         if (cl == MLA_TRACE_CLUSTER && (n) < kTraceTiles) g_mla_trace[r][(n)][(ev)] = global_timer_ns(); \
     } while (0)
-// Per-CTA summary of every cluster: [cluster][rank][8] = entry, after the
+// Per-CTA summary of every cluster: [cluster][rank][24] = entry, after the
 // grid dependency wait, first S issued, last O issued, last epilogue done,
-// exit, tiles, pieces.
+// exit, tiles, pieces, SM id, then clock cycles spent in the barrier waits
+// listed at kTw* (one representative thread per role).
 constexpr int kTraceAllClusters = 256;
-__device__ unsigned long long g_mla_trace_all[kTraceAllClusters][2][8];
+__device__ unsigned long long g_mla_trace_all[kTraceAllClusters][2][24];
+enum {
+    kTwFull,      // S issuer: tile data
+    kTwSFree,     // S issuer: previous S read out of TMEM
+    kTwQFull,     // S issuer: Q-hat of a piece
+    kTwSFull,     // exchange: S complete
+    kTwOwnFree,   // exchange: buffers of tile h-2 released (own and peer)
+    kTwXFull,     // softmax: own and peer partials
+    kTwPFree,     // softmax: P buffer released by O(g-2) (and O ready for a rescale)
+    kTwPFull,     // O issuer: P published
+    kTwOFree,     // O issuer: previous piece's O read
+    kTwEmpty,     // producer: stage released
+    kTwN
+};
+constexpr int kTwBase = 9;
+#define MLA_TW(slot, call) mla_tw_(tw_acc[(slot)], [&]() { return (bool)(call); })
+template <class F>
+__device__ __forceinline__ bool mla_tw_(unsigned long long& acc, F f) {
+    const long long t0 = clock64();
+    const bool ok = f();
+    acc += (unsigned long long)(clock64() - t0);
+    return ok;
+}
 #define MLA_TRACE_ALL(ev, value)                                         \
     do {                                                                 \
         if (cl < kTraceAllClusters) g_mla_trace_all[cl][r][(ev)] = (value); \
@@ -148,6 +173,7 @@ __device__ unsigned long long g_mla_trace_all[kTraceAllClusters][2][8];
 #define MLA_TRACE_ALL(ev, value) \
     do {                         \
     } while (0)
+#define MLA_TW(slot, call) (call)
 #define MLA_TRACE_POINT(ev, n) \
     do {                       \
     } while (0)
@@ -284,6 +310,16 @@ __global__ void __launch_bounds__(kAttThreads, 1)
 
     if (threadIdx.x == 0) MLA_TRACE_POINT(0, kTraceProlog);
     if (threadIdx.x == 0) MLA_TRACE_ALL(0, global_timer_ns());
+#ifdef MLA_TRACE
+    unsigned long long tw_acc[kTwN];
+#pragma unroll
+    for (int i = 0; i < kTwN; ++i) tw_acc[i] = 0;
+    if (threadIdx.x == 0) {
+        unsigned smid;
+        asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+        MLA_TRACE_ALL(8, smid);
+    }
+#endif
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(bar(kBarFull0 + s), 1);
@@ -375,7 +411,7 @@ __global__ void __launch_bounds__(kAttThreads, 1)
                     wp.advance();
                 }
                 const int st = n % kStages;
-                if (n >= kStages && !mbar_wait(bar(kBarEmpty0 + st), ((n / kStages) - 1) & 1)) {
+                if (n >= kStages && !MLA_TW(kTwEmpty, mbar_wait(bar(kBarEmpty0 + st), ((n / kStages) - 1) & 1))) {
                     *abort_flag = 1;
                     break;
                 }
@@ -406,13 +442,13 @@ __global__ void __launch_bounds__(kAttThreads, 1)
         int T_s = ws.valid ? args.seqlens[ws.seq] : 0;  // length of the sequence of tile g
         bool ok = true;
         for (int g = 0; ws.valid && ok && !*abort_flag; ++g) {
-            if (ws.first() && !mbar_wait(bar(kBarQFull), ws.seg & 1)) { ok = false; break; }
+            if (ws.first() && !MLA_TW(kTwQFull, mbar_wait(bar(kBarQFull), ws.seg & 1))) { ok = false; break; }
             const uint32_t tile_off = kOffStages + (g % kStages) * kStageBytes;
-            if (!mbar_wait(bar(kBarFull0 + g % kStages), (g / kStages) & 1)) { ok = false; break; }
+            if (!MLA_TW(kTwFull, mbar_wait(bar(kBarFull0 + g % kStages), (g / kStages) & 1))) { ok = false; break; }
 #ifdef MLA_TRACE
             if (lane == 0) MLA_TRACE_POINT(10, g);
 #endif
-            if (g > 0 && !mbar_wait(bar(kBarSFree), (g - 1) & 1)) { ok = false; break; }
+            if (g > 0 && !MLA_TW(kTwSFree, mbar_wait(bar(kBarSFree), (g - 1) & 1))) { ok = false; break; }
             const int valid = T_s - ws.t * kNk;
             if (valid < kNk) {
                 // Rows at or beyond T_b hold no cached token: zero the latent
@@ -462,8 +498,8 @@ __global__ void __launch_bounds__(kAttThreads, 1)
         wo.init(args.plan, grp);
         bool ok = true;
         for (int g = 0; wo.valid && ok && !*abort_flag; ++g, wo.advance()) {
-            if (!mbar_wait(bar(kBarPFull0 + (g & 1)), (g >> 1) & 1)) { ok = false; break; }
-            if (wo.first() && wo.seg > 0 && !mbar_wait(bar(kBarOFree), (wo.seg - 1) & 1)) { ok = false; break; }
+            if (!MLA_TW(kTwPFull, mbar_wait(bar(kBarPFull0 + (g & 1)), (g >> 1) & 1))) { ok = false; break; }
+            if (wo.first() && wo.seg > 0 && !MLA_TW(kTwOFree, mbar_wait(bar(kBarOFree), (wo.seg - 1) & 1))) { ok = false; break; }
             tc_fence_after();
             if (lane == 0) {
                 MLA_TRACE_POINT(15, g);
@@ -530,7 +566,7 @@ __global__ void __launch_bounds__(kAttThreads, 1)
         for (int h = 0; w.valid && ok && !*abort_flag; ++h, w.advance()) {
             const int hb = h & 1;
             // ---- partial S(h) of this half, in log2 units, rounded to fp16
-            if (!mbar_wait(bar(kBarSFull), h & 1)) { ok = false; break; }
+            if (!MLA_TW(kTwSFull, mbar_wait(bar(kBarSFull), h & 1))) { ok = false; break; }
             tc_fence_after();
             uint32_t own[32];
             {
@@ -552,8 +588,8 @@ __global__ void __launch_bounds__(kAttThreads, 1)
             // ---- publish: Own[hb] (read by our softmax warps and by the bulk copy
             // into the peer's X[hb]); both readers of tile h-2 must be done.
             if (h >= 2) {
-                if (!mbar_wait(bar(kBarOwnFree0 + hb), ((h >> 1) - 1) & 1)) { ok = false; break; }
-                if (!mbar_wait_cluster(bar(kBarXFree0 + hb), ((h >> 1) - 1) & 1)) { ok = false; break; }
+                if (!MLA_TW(kTwOwnFree, mbar_wait(bar(kBarOwnFree0 + hb), ((h >> 1) - 1) & 1))) { ok = false; break; }
+                if (!MLA_TW(kTwOwnFree, mbar_wait_cluster(bar(kBarXFree0 + hb), ((h >> 1) - 1) & 1))) { ok = false; break; }
             }
             const uint32_t own_buf = base + kOffOwn + hb * kXBytes;
 #pragma unroll
@@ -597,8 +633,8 @@ __global__ void __launch_bounds__(kAttThreads, 1)
         for (int g = 0; w.valid && ok && !*abort_flag; ++g, w.advance()) {
             const int b2 = g & 1;
             // ---- S(g) for this thread's 32 keys = own partial + the peer's (same order on both CTAs)
-            if (!mbar_wait(bar(kBarOwnFull0 + b2), (g >> 1) & 1)) { ok = false; break; }
-            if (!mbar_wait_cluster(bar(kBarXFull0 + b2), (g >> 1) & 1)) { ok = false; break; }
+            if (!MLA_TW(kTwXFull, mbar_wait(bar(kBarOwnFull0 + b2), (g >> 1) & 1))) { ok = false; break; }
+            if (!MLA_TW(kTwXFull, mbar_wait_cluster(bar(kBarXFull0 + b2), (g >> 1) & 1))) { ok = false; break; }
             float s[32];
             {
                 const uint32_t own_buf = base + kOffOwn + b2 * kXBytes;
@@ -662,11 +698,11 @@ __global__ void __launch_bounds__(kAttThreads, 1)
             }
             if (threadIdx.x == 64) MLA_TRACE_POINT(9, g);
             // P buffer b2 was last read by O(g-2).
-            if (g >= 2 && !mbar_wait(bar(kBarPFree0 + b2), ((g >> 1) - 1) & 1)) { ok = false; break; }
+            if (g >= 2 && !MLA_TW(kTwPFree, mbar_wait(bar(kBarPFree0 + b2), ((g >> 1) - 1) & 1))) { ok = false; break; }
             if (grow) {
                 if (!first) {
                     // O must hold everything up to tile g-1 before it is rescaled.
-                    if (!mbar_wait(bar(kBarPFree0 + (b2 ^ 1)), ((g - 1) >> 1) & 1)) { ok = false; break; }
+                    if (!MLA_TW(kTwPFree, mbar_wait(bar(kBarPFree0 + (b2 ^ 1)), ((g - 1) >> 1) & 1))) { ok = false; break; }
                     tc_fence_after();
                     const float f = ex2(m_used - mx);
                     l_part *= f;
@@ -767,6 +803,13 @@ __global__ void __launch_bounds__(kAttThreads, 1)
         if (!ok) *abort_flag = 1;
     }
 
+#ifdef MLA_TRACE
+    if (threadIdx.x == 0 || threadIdx.x == 32 || threadIdx.x == 64 || threadIdx.x == 192 || threadIdx.x == 320) {
+#pragma unroll
+        for (int i = 0; i < kTwN; ++i)
+            if (tw_acc[i]) MLA_TRACE_ALL(kTwBase + i, tw_acc[i]);
+    }
+#endif
     if (*abort_flag && threadIdx.x == 0) atomicOr(args.status, MLA_STATUS_TIMEOUT);
     tc_fence_before();
     __syncthreads();
@@ -794,7 +837,7 @@ __device__ __forceinline__ void mla_plan_warp(const int32_t* __restrict__ seqlen
     int* splits = pre + B + 1;
     const int groups = clusters / q_len > 0 ? clusters / q_len : 1;
     for (int g = lane; g < groups; g += 32) gfirst[g] = B;
-    int carry = 0;
+    int carry = 0, c_min = INT_MAX, c_max = 0;
     if (lane == 0) pre[0] = 0;
     for (int base = 0; base < B; base += 32) {
         const int b = base + lane;
@@ -803,6 +846,8 @@ __device__ __forceinline__ void mla_plan_warp(const int32_t* __restrict__ seqlen
             const int T = seqlens[b];
             if (T < q_len || T > T_max) atomicOr(status, MLA_STATUS_BAD_SEQLEN);
             else c = (T + kNk - 1) / kNk + ovh;
+            c_min = min(c_min, c);
+            c_max = max(c_max, c);
         }
         int v = c;
 #pragma unroll
@@ -814,6 +859,19 @@ __device__ __forceinline__ void mla_plan_warp(const int32_t* __restrict__ seqlen
         carry += __shfl_sync(0xffffffffu, v, 31);
     }
     int L = (carry + groups - 1) / groups;
+    // A batch of equal, valid lengths may be cut at sequence boundaries
+    // instead: no partials and no combine pass, which costs more than a few
+    // tiles per group; taken when the whole-sequence share is within a quarter
+    // of the even share.
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        c_min = min(c_min, __shfl_xor_sync(0xffffffffu, c_min, o));
+        c_max = max(c_max, __shfl_xor_sync(0xffffffffu, c_max, o));
+    }
+    if (c_min == c_max && c_max > 0) {
+        const int whole = ((B + groups - 1) / groups) * c_max;
+        if (whole <= L + L / 4) L = whole;
+    }
     if (L < min_units) L = min_units;
     if (L < 1) L = 1;
     __syncwarp();

@@ -89,6 +89,8 @@ SMALL_CASES = [
     ((3000, 2, 900) * 3, 2, 0),   # ragged verify batch
     ((1500, 9, 260), 8, 0),       # long verify window: 8 query tokens per sequence
     ((16, 700), 16, 5),           # the largest q_len; the first sequence holds only its new tokens
+    ((640,) * 7, 1, 8),           # equal lengths: one whole sequence per cluster, one cluster idle
+    ((256,) * 7, 2, 8),           # equal lengths: two whole sequences per cluster group
 ]
 
 
