@@ -23,6 +23,17 @@ extern "C" int mla_trace_read(void* host, size_t bytes) {
 extern "C" int mla_trace_read_all(void* host, size_t bytes) {
     return cudaMemcpyFromSymbol(host, mla::sm100::g_mla_trace_all, bytes) == cudaSuccess ? 0 : -4;
 }
+extern "C" int mla_trace_read_kt(void* host, size_t bytes) {
+    return cudaMemcpyFromSymbol(host, mla::sm100::g_mla_ktrace, bytes) == cudaSuccess ? 0 : -4;
+}
+extern "C" int mla_trace_clear_kt(void) {
+    unsigned long long init[mla::sm100::kKtN][3];
+    for (int k = 0; k < mla::sm100::kKtN; ++k) {
+        init[k][0] = init[k][1] = ~0ull;
+        init[k][2] = 0;
+    }
+    return cudaMemcpyToSymbol(mla::sm100::g_mla_ktrace, init, sizeof(init)) == cudaSuccess ? 0 : -4;
+}
 extern "C" int mla_trace_clear(void) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, mla::sm100::g_mla_trace) != cudaSuccess) return -4;
@@ -77,6 +88,7 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64
 __global__ void append_v3_kernel(const __nv_bfloat16* __restrict__ c_kv, const __nv_bfloat16* __restrict__ k_rope,
                                  const int32_t* __restrict__ pos, int B, int n_tok, CacheView cache, RopeTable rope,
                                  int* status) {
+    MLA_KT(kKtAppend, 0);
     const int gw = (blockIdx.x * blockDim.x + threadIdx.x) / 32;
     const int lane = threadIdx.x & 31;
     if (gw >= B * n_tok) return;
@@ -96,6 +108,7 @@ __global__ void append_v3_kernel(const __nv_bfloat16* __restrict__ c_kv, const _
     float y0, y1;
     mla_rope_rotate(__low2float(k2), __high2float(k2), rope.inv_freq[lane], t, &y0, &y1);
     reinterpret_cast<__nv_bfloat162*>(row + kLat)[lane] = __floats2bfloat162_rn(y0, y1);
+    MLA_KT(kKtAppend, 2);
 }
 
 // Opt a kernel into more than 48 KB of dynamic shared memory, once per device

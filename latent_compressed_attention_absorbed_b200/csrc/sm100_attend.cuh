@@ -32,18 +32,21 @@
 // groups writes fp32 partials plus a base-2 LSE per head and token, merged by
 // the combine kernel.
 //
-// Roles per CTA (352 threads):
+// Roles per CTA (512 threads; warps 12-15 are the second softmax warp of each
+// quarter, warp 11 is idle):
 //   warp 0     TMA producer (stage ring, L2 prefetch of the tiles ahead);
 //   warp 1     TMEM owner and issuer of the score MMAs (S);
 //   warp 10    issuer of the P.V MMAs (O), as soon as P is published;
-//   warps 2-5  softmax: add the two partial scores, online softmax, P into
-//              TMEM, rescale / normalise O, write o_lat or split partials;
+//   warps 2-5, softmax, two warps per TMEM lane quarter (32 keys each): add
+//   12-15      the two partial scores, online softmax, P into TMEM, rescale /
+//              normalise O, write o_lat or split partials;
 //   warps 6-9  exchange: read partial S out of TMEM, publish it (local copy
 //              for the softmax warps, bulk copy to the peer), load Q-hat.
 // Warp w reaches TMEM lanes 32*(w%4)..+31; lane l of warp w owns head
 // 32*(w%4)+l, a whole score row.  Every wait is bounded; on expiry the
 // kernel flags MLA_STATUS_TIMEOUT, stops issuing work and tears down
-// normally.
+// normally (the two softmax warps of a quarter, which meet on a named
+// barrier, decide together whether to stop, so neither is left waiting).
 #pragma once
 
 #include <cuda_bf16.h>
@@ -88,7 +91,8 @@ constexpr int kOffX = kOffOwn + 2 * kXBytes;
 constexpr int kQRBytes = kHeads * 64;                  // 8192
 constexpr int kOffQR = kOffX + 2 * kXBytes;
 constexpr int kOffRed = kOffQR + kQRBytes;            // softmax pair exchange: [2][2][128] fp32
-constexpr int kOffBars = kOffRed + 2 * 2 * kHeads * 4;
+constexpr int kOffFlags = kOffRed + 2 * 2 * kHeads * 4;  // softmax pair status: [2][4 quarters][2] int
+constexpr int kOffBars = kOffFlags + 2 * 4 * 2 * 4;
 constexpr int kAttSmem = kOffBars + 256 + 1024;
 static_assert(kAttSmem <= 232448, "attention kernel shared memory exceeds 227 KB");
 
@@ -114,7 +118,7 @@ enum {
     kBarXFull0 = kBarOwnFree0 + 2,     // peer's partial g landed in X[g%2] (tx)
     kBarXFree0 = kBarXFull0 + 2,       // the peer has read what we sent into its X[g%2] (4, remote)
     kBarOFull = kBarXFree0 + 2,        // last O of a piece complete (MMA commit)
-    kBarOFree,                         // O read by the epilogue (4 softmax warps)
+    kBarOFree,                         // O read by the epilogue (8 softmax warps)
     kNumBars
 };
 static_assert(8 * (kNumBars + 2) <= 256, "barrier block too small");
@@ -157,7 +161,11 @@ enum {
     kTwN
 };
 constexpr int kTwBase = 9;
+#ifdef MLA_TRACE_WAITS
 #define MLA_TW(slot, call) mla_tw_(tw_acc[(slot)], [&]() { return (bool)(call); })
+#else
+#define MLA_TW(slot, call) (call)
+#endif
 template <class F>
 __device__ __forceinline__ bool mla_tw_(unsigned long long& acc, F f) {
     const long long t0 = clock64();
@@ -169,7 +177,21 @@ __device__ __forceinline__ bool mla_tw_(unsigned long long& acc, F f) {
     do {                                                                 \
         if (cl < kTraceAllClusters) g_mla_trace_all[cl][r][(ev)] = (value); \
     } while (0)
+// Kernel timeline of the decode step: [kernel][first entry, first return
+// from the grid dependency wait, last exit], stamped by thread 0 of each CTA.
+enum { kKtAppend, kKtAbsorb, kKtAttend, kKtCombine, kKtProject, kKtN };
+__device__ unsigned long long g_mla_ktrace[kKtN][3];
+#define MLA_KT(k, ev)                                                                       \
+    do {                                                                                    \
+        if (threadIdx.x == 0) {                                                             \
+            if ((ev) < 2) atomicMin(&::mla::sm100::g_mla_ktrace[k][ev], global_timer_ns()); \
+            else atomicMax(&::mla::sm100::g_mla_ktrace[k][ev], global_timer_ns());          \
+        }                                                                                   \
+    } while (0)
 #else
+#define MLA_KT(k, ev) \
+    do {              \
+    } while (0)
 #define MLA_TRACE_ALL(ev, value) \
     do {                         \
     } while (0)
@@ -310,10 +332,13 @@ __global__ void __launch_bounds__(kAttThreads, 1)
 
     if (threadIdx.x == 0) MLA_TRACE_POINT(0, kTraceProlog);
     if (threadIdx.x == 0) MLA_TRACE_ALL(0, global_timer_ns());
-#ifdef MLA_TRACE
+    MLA_KT(kKtAttend, 0);
+#ifdef MLA_TRACE_WAITS
     unsigned long long tw_acc[kTwN];
 #pragma unroll
     for (int i = 0; i < kTwN; ++i) tw_acc[i] = 0;
+#endif
+#ifdef MLA_TRACE
     if (threadIdx.x == 0) {
         unsigned smid;
         asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
@@ -361,6 +386,7 @@ __global__ void __launch_bounds__(kAttThreads, 1)
     if (threadIdx.x == 0) pdl_trigger();
     if (threadIdx.x == 0) MLA_TRACE_POINT(2, kTraceProlog);
     if (threadIdx.x == 0) MLA_TRACE_ALL(1, global_timer_ns());
+    MLA_KT(kKtAttend, 1);
     const bool active = grp < args.plan->groups;
     // Warp 0, lanes 1..31: spread the optional L2 prefetch over the grid, 16 KB a request.
     if (warp == 0 && lane > 0 && args.prefetch) {
@@ -621,22 +647,30 @@ __global__ void __launch_bounds__(kAttThreads, 1)
         // ======================================================== softmax warps 2..5 and 12..15
         // Two warps per TMEM quarter: half kh takes keys 32kh..32kh+31 of each
         // score row and latent columns 128kh..128kh+127 of O; the pair agrees on
-        // the row maximum through shared memory (named barrier 1 + quarter).
+        // the row maximum through shared memory, meeting on named barrier
+        // 1 + quarter.  Both warps walk the same tiles and meet at the same
+        // points; a failed (timed-out) wait does not leave the loop at once: the
+        // warp skips the tile's side effects up to the next meeting, where both
+        // read each other's status and stop together (a hardware barrier has no
+        // time limit, so neither may wait at one the other never reaches).
         const int kh = warp >= 12 ? 1 : 0;
         const uint32_t xfree_peer = mapa(bar(kBarXFree0), peer);
         float* red = reinterpret_cast<float*>(base_ptr + kOffRed);  // [2 tiles][2 halves][128 rows]
+        volatile int* pair_ok = reinterpret_cast<volatile int*>(base_ptr + kOffFlags);
         bool ok = true;
         TileWalk w;
         w.init(args.plan, grp);
         float m_used = -CUDART_INF_F, l_part = 0.f;
         int n_keys = 0;
-        for (int g = 0; w.valid && ok && !*abort_flag; ++g, w.advance()) {
+        for (int g = 0; w.valid; ++g, w.advance()) {
             const int b2 = g & 1;
             // ---- S(g) for this thread's 32 keys = own partial + the peer's (same order on both CTAs)
-            if (!MLA_TW(kTwXFull, mbar_wait(bar(kBarOwnFull0 + b2), (g >> 1) & 1))) { ok = false; break; }
-            if (!MLA_TW(kTwXFull, mbar_wait_cluster(bar(kBarXFull0 + b2), (g >> 1) & 1))) { ok = false; break; }
+            if (ok) ok = MLA_TW(kTwXFull, mbar_wait(bar(kBarOwnFull0 + b2), (g >> 1) & 1));
+            if (ok) ok = MLA_TW(kTwXFull, mbar_wait_cluster(bar(kBarXFull0 + b2), (g >> 1) & 1));
             float s[32];
-            {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) s[j] = 0.f;
+            if (ok) {
                 const uint32_t own_buf = base + kOffOwn + b2 * kXBytes;
                 const uint32_t x_buf = base + kOffX + b2 * kXBytes;
 #pragma unroll
@@ -658,7 +692,7 @@ __global__ void __launch_bounds__(kAttThreads, 1)
             // Both buffers are consumed (their values are in registers and used
             // by the adds above), so relaxed arrives suffice.
             __syncwarp();
-            if (lane == 0) {
+            if (ok && lane == 0) {
                 mbar_arrive(bar(kBarOwnFree0 + b2));
                 mbar_arrive_remote_relaxed(xfree_peer + 8 * b2);
             }
@@ -680,7 +714,13 @@ __global__ void __launch_bounds__(kAttThreads, 1)
             }
             float* rg = red + (b2 * 2) * kHeads;  // this tile's [2 halves][128 rows]
             rg[kh * kHeads + m] = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+            volatile int* st_pair = pair_ok + (b2 * 4 + quarter) * 2;  // this tile's status of the pair
+            if (lane == 0) st_pair[kh] = (ok && !*abort_flag) ? 1 : 0;
             named_bar_sync(1 + quarter, 64);
+            if (!st_pair[0] || !st_pair[1]) {
+                ok = false;
+                break;
+            }
             const float mx = fmaxf(rg[m], rg[kHeads + m]);
             if (threadIdx.x == 64) MLA_TRACE_POINT(8, g);
             const bool first = w.first();
@@ -697,12 +737,15 @@ __global__ void __launch_bounds__(kAttThreads, 1)
                 pk[j] = pack_bf16(p0, p1);
             }
             if (threadIdx.x == 64) MLA_TRACE_POINT(9, g);
-            // P buffer b2 was last read by O(g-2).
-            if (g >= 2 && !MLA_TW(kTwPFree, mbar_wait(bar(kBarPFree0 + b2), ((g >> 1) - 1) & 1))) { ok = false; break; }
-            if (grow) {
+            // P buffer b2 was last read by O(g-2).  (From here to the next
+            // meeting a failed wait only skips work.)
+            if (g >= 2 && ok) ok = MLA_TW(kTwPFree, mbar_wait(bar(kBarPFree0 + b2), ((g >> 1) - 1) & 1));
+            if (grow && ok) {
                 if (!first) {
                     // O must hold everything up to tile g-1 before it is rescaled.
-                    if (!MLA_TW(kTwPFree, mbar_wait(bar(kBarPFree0 + (b2 ^ 1)), ((g - 1) >> 1) & 1))) { ok = false; break; }
+                    ok = MLA_TW(kTwPFree, mbar_wait(bar(kBarPFree0 + (b2 ^ 1)), ((g - 1) >> 1) & 1));
+                }
+                if (ok && !first) {
                     tc_fence_after();
                     const float f = ex2(m_used - mx);
                     l_part *= f;
@@ -718,13 +761,15 @@ __global__ void __launch_bounds__(kAttThreads, 1)
                 }
                 m_used = mx;
             }
-            tc_fence_after();
-            l_part += rs0 + rs1;
-            tmem_st16(tmem + lane_addr + kTmemP + 32 * b2 + 16 * kh, pk);
-            tmem_wait_st();
-            tc_fence_before();
+            if (ok) {
+                tc_fence_after();
+                l_part += rs0 + rs1;
+                tmem_st16(tmem + lane_addr + kTmemP + 32 * b2 + 16 * kh, pk);
+                tmem_wait_st();
+                tc_fence_before();
+            }
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(kBarPFull0 + b2));
+            if (ok && lane == 0) mbar_arrive(bar(kBarPFull0 + b2));
             if (threadIdx.x == 64) MLA_TRACE_POINT(6, g);
 #ifndef MLA_TRACE_CYCLES
             if (threadIdx.x == 96) MLA_TRACE_POINT(11, g);
@@ -732,14 +777,17 @@ __global__ void __launch_bounds__(kAttThreads, 1)
 #endif
             if (threadIdx.x == 160) MLA_TRACE_POINT(13, g);
             // ---- epilogue at the end of a piece: this thread owns O row m, columns 128kh..+127
+            float l_sum = 0.f;
             if (w.last()) {
                 // the row's softmax denominator: both halves' partial sums
                 float* rl = red + (b2 * 2) * kHeads;
                 named_bar_sync(1 + quarter, 64);  // the pair has read this tile's maxima
                 rl[kh * kHeads + m] = l_part;
                 named_bar_sync(1 + quarter, 64);
-                const float l_sum = rl[m] + rl[kHeads + m];
-                if (!mbar_wait(bar(kBarOFull), w.seg & 1)) { ok = false; break; }
+                l_sum = rl[m] + rl[kHeads + m];
+                if (ok) ok = mbar_wait(bar(kBarOFull), w.seg & 1);
+            }
+            if (w.last() && ok) {
                 tc_fence_after();
                 const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
                 const int u = w.seq * q_len + qi;
@@ -803,7 +851,7 @@ __global__ void __launch_bounds__(kAttThreads, 1)
         if (!ok) *abort_flag = 1;
     }
 
-#ifdef MLA_TRACE
+#ifdef MLA_TRACE_WAITS
     if (threadIdx.x == 0 || threadIdx.x == 32 || threadIdx.x == 64 || threadIdx.x == 192 || threadIdx.x == 320) {
 #pragma unroll
         for (int i = 0; i < kTwN; ++i)
@@ -820,6 +868,7 @@ __global__ void __launch_bounds__(kAttThreads, 1)
     cluster_sync();
     if (threadIdx.x == 0) MLA_TRACE_POINT(7, kTraceProlog);
     if (threadIdx.x == 0) MLA_TRACE_ALL(5, global_timer_ns());
+    MLA_KT(kKtAttend, 2);
 }
 
 // ------------------------------------------------------------------ plan
@@ -1021,11 +1070,16 @@ __global__ void __launch_bounds__(256) mla_combine_kernel(const Plan* __restrict
                                                           const float* __restrict__ part_o,
                                                           const float* __restrict__ part_lse,
                                                           __nv_bfloat16* __restrict__ o_lat) {
+    MLA_KT(kKtCombine, 0);
     pdl_wait();
     pdl_trigger();
+    MLA_KT(kKtCombine, 1);
     const int q_len = plan->q_len;
     const int work = blockIdx.x / (kHeads / 8);
-    if (work >= plan->n_split * q_len) return;
+    if (work >= plan->n_split * q_len) {
+        MLA_KT(kKtCombine, 2);
+        return;
+    }
     const int lane = threadIdx.x % 32;
     const int h = (blockIdx.x % (kHeads / 8)) * 8 + threadIdx.x / 32;
     const int b = plan_splits(plan)[work / q_len];
@@ -1044,6 +1098,7 @@ __global__ void __launch_bounds__(256) mla_combine_kernel(const Plan* __restrict
         o.y = pack_bf16(ms.acc[j].z, ms.acc[j].w);
         dst[32 * j] = o;
     }
+    MLA_KT(kKtCombine, 2);
 }
 
 }  // namespace sm100

@@ -73,6 +73,7 @@ __global__ void __launch_bounds__(128, 1)
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int h = blockIdx.x;
     const int n0 = blockIdx.y * NT;
+    MLA_KT(ROPE ? kKtAbsorb : kKtProject, 0);
     const int m0 = blockIdx.z * 128;
 
     if (threadIdx.x == 0) {
@@ -153,6 +154,7 @@ __global__ void __launch_bounds__(128, 1)
     }
     // Nothing is written before the kernels this one depends on have completed.
     pdl_wait();
+    MLA_KT(ROPE ? kKtAbsorb : kKtProject, 1);
     if (warp == 2 && args.plan && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0)
         mla_plan_warp(args.seqlens, args.plan_B, args.q_len, args.plan_T_max, args.plan_clusters, args.plan_ovh,
                       args.plan_min_units, args.plan, args.status, args.plan_olat, lane);
@@ -230,6 +232,7 @@ __global__ void __launch_bounds__(128, 1)
     tc_fence_before();
     __syncthreads();
     if (warp == 1) tmem_dealloc(tmem, C::kTmemCols);
+    MLA_KT(ROPE ? kKtAbsorb : kKtProject, 2);
 }
 
 }  // namespace sm100

@@ -71,12 +71,14 @@ __global__ void __launch_bounds__(128) absorb_gemv_kernel(AbsorbGemvArgs a) {
     auto w_s = reinterpret_cast<__nv_bfloat16(*)[256]>(gemv_smem);                 // W_UK[h][d][256y ..]
     auto q_s = reinterpret_cast<float(*)[128]>(gemv_smem + kGemvWBytes);          // q_nope rows, fp32
     const int h = blockIdx.x, y = blockIdx.y, t = threadIdx.x;
+    MLA_KT(kKtAbsorb, 0);
     if (h == kHeads) {
         pdl_wait();
         if (y == 0 && t < 32 && a.plan)
             mla_plan_warp(a.seqlens, a.plan_B, a.q_len, a.plan_T_max, a.plan_clusters, a.plan_ovh,
                           a.plan_min_units, a.plan, a.status, a.plan_olat, t);
         if (t == 0) pdl_trigger();
+        MLA_KT(kKtAbsorb, 2);
         return;
     }
     // weights first (they do not depend on the previous kernel): 128 rows x 512 B
@@ -91,6 +93,7 @@ __global__ void __launch_bounds__(128) absorb_gemv_kernel(AbsorbGemvArgs a) {
     }
     pdl_wait();
     if (t == 0) pdl_trigger();
+    MLA_KT(kKtAbsorb, 1);
     for (int i = t; i < R * 128; i += 128) {
         const int u = i / 128, d = i % 128;
         q_s[u][d] = u < a.rows ? __bfloat162float(a.q_nope[((size_t)u * kHeads + h) * 128 + d]) : 0.f;
@@ -130,6 +133,7 @@ __global__ void __launch_bounds__(128) absorb_gemv_kernel(AbsorbGemvArgs a) {
         if (u < a.rows)
             reinterpret_cast<__nv_bfloat162*>(a.q_hat + ((size_t)u * kHeads + h) * kRow + 256 * y)[t] =
                 __floats2bfloat162_rn(acc[u][0], acc[u][1]);
+    MLA_KT(kKtAbsorb, 2);
 }
 
 struct ProjectGemvArgs {
@@ -163,6 +167,7 @@ __global__ void __launch_bounds__(512) project_gemv_kernel(ProjectGemvArgs a) {
     const int h = blockIdx.x, t = threadIdx.x;
     const int warp = t / 32, lane = t % 32;
     const int u = warp % R, g = warp / R;
+    MLA_KT(kKtProject, 0);
     {
         const uint32_t ws = smem_u32(w_s);
         const __nv_bfloat16* src = a.W_UV + (size_t)h * 128 * kLat;
@@ -174,6 +179,7 @@ __global__ void __launch_bounds__(512) project_gemv_kernel(ProjectGemvArgs a) {
     }
     pdl_wait();
     if (t == 0) pdl_trigger();
+    MLA_KT(kKtProject, 1);
     // ---- 1. o_lat of row u
     bool split = false;
     UnitPieces up;
@@ -262,6 +268,7 @@ __global__ void __launch_bounds__(512) project_gemv_kernel(ProjectGemvArgs a) {
             a.out[((size_t)uu * kHeads + h) * 128 + v] =
                 __float2bfloat16_rn(sum_s[0][uu][v] + sum_s[1][uu][v] + sum_s[2][uu][v] + sum_s[3][uu][v]);
     }
+    MLA_KT(kKtProject, 2);
 }
 
 }  // namespace sm100

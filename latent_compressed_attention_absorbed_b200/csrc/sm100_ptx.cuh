@@ -389,6 +389,8 @@ __device__ __forceinline__ void ld_shared_v4f(uint32_t addr, float& a, float& b,
                  : "memory");
 }
 
+// Named barrier `id` for `nthreads` threads (a multiple of 32).  It has no time
+// limit: callers must reach it the same number of times.
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
