@@ -115,8 +115,10 @@ size_t mla_workspace_bytes(const mla_dims_t* dims, int32_t B, int32_t q_len);
  *   W_UK   [H][d_n][d_c]        k_C = W_UK[h] c      (U in R^{d_h x d_c})
  *   W_UV   [H][d_v][d_c]        v   = W_UV[h] c
  *   out    [B][q_len][H][d_v]   written
- *   workspace: device scratch of at least mla_workspace_bytes(); the call
- *   owns it until the stream reaches the end of the call.
+ *   workspace: device scratch of at least mla_workspace_bytes(), 16-byte
+ *   aligned; the library rounds its base up to 256 bytes inside the buffer
+ *   (mla_workspace_bytes() includes that slack).  The call owns it until the
+ *   stream reaches the end of the call.
  * Steps: absorb (a2), attend in latent space (a3+a4), project (a5). */
 int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_rope,
                const void* W_UK, const void* W_UV, const mla_cache_t* cache,
@@ -127,12 +129,16 @@ int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_rope,
  *   path: 0 = auto (sm_100a tensor-core kernels for bf16 V3 geometry, generic
  *         CUDA kernels otherwise), 1 = force the tensor-core path
  *         (MLA_ERR_UNSUPPORTED if it cannot run), 2 = force the generic path.
- *   num_pairs: CTA pairs (clusters) of the attention grid (0 = one per two SMs).
+ *   num_pairs: CTA pairs (clusters) of the attention grid (0 = one per two SMs;
+ *         at most 1024).
  *   overhead_tiles: scheduling cost charged per query token (each of the
  *         B * q_len tokens is scheduled on its own), in 64-key tiles
- *         (negative = default).
+ *         (negative = default, 2).
  *   min_tiles: smallest piece of a token's keys one cluster takes, in 64-key tiles
- *         (0 = default); larger values mean fewer split partials to merge.
+ *         (0 = default, 2); larger values mean fewer split partials to merge.
+ *         A batch whose sequences all have the same length is cut at sequence
+ *         boundaries when that costs at most a quarter more per cluster group
+ *         than an even split.
  *   events / n_events: optional caller-created cudaEvent_t handles; when
  *         n_events >= MLA_NUM_EVENTS, mla_decode_ex records them on `stream`
  *         at the stage boundaries listed below, so a caller can time each
