@@ -359,8 +359,8 @@ def run_reference(args):
     cb["value"] = round(v, 1)
     line = {"impl": "reference", "metric": metric_name(), "value": round(v, 1), "unit": "us/step", "n_gpus": 0,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(v / 1e3, 3), "higher_is_better": False,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded, BASELINE value "
-            "distributions)", "config": config_of(cfg, args), "cpu_baseline": cb,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded; c_KV, k_R, q ~ N(0,1), "
+            "W ~ N(0,0.02))", "config": config_of(cfg, args), "cpu_baseline": cb,
             "e2e": {"value": round(v, 1), "unit": "us/step", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
