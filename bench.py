@@ -96,6 +96,26 @@ def traffic_for(workload, kernel):
 
 # ------------------------------------------------------------------ clocks
 
+def nvml_handle(nv, props, index):
+    """NVML handle of the CUDA device `index` described by `props`, and how it
+    was matched.  NVML numbers the GPUs of the host, ignoring
+    CUDA_VISIBLE_DEVICES, so the device is matched by UUID, then by PCI
+    address, and by index only as a last resort."""
+    uuid = str(getattr(props, "uuid", "") or "") if props is not None else ""
+    if uuid:
+        try:
+            return nv.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid), "uuid"
+        except Exception:
+            pass
+    if props is not None and hasattr(props, "pci_bus_id"):
+        bus = f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
+        try:
+            return nv.nvmlDeviceGetHandleByPciBusId(bus), "pci"
+        except Exception:
+            pass
+    return nv.nvmlDeviceGetHandleByIndex(index), "index"
+
+
 class ClockSampler:
     """Samples SM clock and throttle reasons with NVML during the timed region."""
 
@@ -103,14 +123,15 @@ class ClockSampler:
                0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
                0x100: "display_clock_setting"}
 
-    def __init__(self, index, period=0.01):
+    def __init__(self, index, props=None, period=0.01):
         self.samples, self.reasons, self.period = [], set(), period
         self._stop = threading.Event()
+        self.match = None
         try:
             import pynvml
             pynvml.nvmlInit()
             self.nv = pynvml
-            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.h, self.match = nvml_handle(pynvml, props, index)
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
         except Exception:
             self.nv = None
@@ -143,7 +164,8 @@ class ClockSampler:
         if not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
         return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples),
+                "nvml_match": self.match}
 
 
 # ------------------------------------------------------------------ our arm
@@ -228,7 +250,7 @@ def run_ours(args, rank, world, local_rank):
     # ---- timed: K graph replays, each bracketed by events, L2 flushed before each
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    with ClockSampler(local_rank) as clk:
+    with ClockSampler(local_rank, torch.cuda.get_device_properties(device)) as clk:
         torch.cuda.synchronize()
         for i in range(args.steps):
             busy()

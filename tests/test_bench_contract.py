@@ -34,3 +34,38 @@ def test_reference_arm_prints_one_contract_line():
 
 def test_reference_arm_prints_nothing_on_other_ranks():
     assert _run({"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"}) == []
+
+
+class _FakeNvml:
+    """Host GPUs 0..2 (NVML numbering); CUDA sees only the one with bus 0x3B."""
+
+    def __init__(self, fail_uuid=False):
+        self.fail_uuid = fail_uuid
+
+    def nvmlDeviceGetHandleByUUID(self, u):
+        if self.fail_uuid or u != "GPU-0000-feed":
+            raise RuntimeError("not found")
+        return "gpu1"
+
+    def nvmlDeviceGetHandleByPciBusId(self, bus):
+        if bus != "00000000:3B:00.0":
+            raise RuntimeError("not found")
+        return "gpu1"
+
+    def nvmlDeviceGetHandleByIndex(self, i):
+        return f"gpu{i}"
+
+
+class _Props:
+    uuid = "0000-feed"
+    pci_domain_id, pci_bus_id, pci_device_id = 0, 0x3B, 0
+
+
+def test_clock_sampler_watches_the_gpu_cuda_runs_on():
+    sys.path.insert(0, ROOT)
+    import bench
+
+    # CUDA device 0 is host GPU 1: matched by UUID, else by PCI address, never by index 0
+    assert bench.nvml_handle(_FakeNvml(), _Props(), 0) == ("gpu1", "uuid")
+    assert bench.nvml_handle(_FakeNvml(fail_uuid=True), _Props(), 0) == ("gpu1", "pci")
+    assert bench.nvml_handle(_FakeNvml(), None, 0) == ("gpu0", "index")
