@@ -139,7 +139,7 @@ def decode_expanded(q_nope: np.ndarray, q_rope: np.ndarray, W_UK: np.ndarray, W_
         T = c.shape[0]
         if T < q_len:
             raise ValueError("a sequence must already hold its q_len new tokens")
-        k_rot = rope(k_raw, np.arange(T))  # key j rotated at its own position j
+        k_rot = rope(k_raw, np.arange(T), base)  # key j rotated at its own position j
         for h in heads:
             K = np.concatenate([c @ W_UK[h].T, k_rot], axis=1)  # [T, d_n + d_r]
             V = c @ W_UV[h].T  # [T, d_v]
@@ -177,7 +177,7 @@ def decode_absorbed(q_nope: np.ndarray, q_rope: np.ndarray, W_UK: np.ndarray, W_
         c, k_raw = histories[b]
         c = np.asarray(c, dtype=np.float64)
         T = c.shape[0]
-        k_rot = rope(k_raw, np.arange(T))
+        k_rot = rope(k_raw, np.arange(T), base)
         for i in range(q_len):
             m = T - q_len + i
             q_lat = np.einsum("hdc,hd->hc", W_UK, q_nope[b, i])  # W_UK[h]^T q_nope, [H, d_c]

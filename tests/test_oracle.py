@@ -150,6 +150,49 @@ def test_hand_derived_two_key_example():
     assert abs(out_a[0, 0, 0, 0] - expect) < 1e-14
 
 
+def test_hand_derived_rope_base_applies_to_keys_and_queries():
+    # Decoupled RoPE rotates q^R and k^R alike (m.lsln.cn/news/222502 section 2.3),
+    # so a non-default base must turn the keys too.  H=1, d_c=d_n=d_v=1, d_r=4,
+    # T=2, q_len=1 (query at position 1), content branch off (W_UK = 0).
+    # Only RoPE pair 1 is used; it turns by pos * base**(-1/2) (pair 0 by pos,
+    # whatever the base).  k_R = (0,0,1,0) at positions 0 and 1 -> (0,0,1,0) and
+    # (0,0,cos a,sin a); q_R = (0,0,1,0) at position 1 -> (0,0,cos a,sin a), with
+    # a = base**-0.5.  RoPE scores: cos a and 1.  Scale 1/sqrt(d_n + d_r) = 1/sqrt(5).
+    base = 500.0
+    a = base ** -0.5
+    W_UK = np.zeros((1, 1, 1))
+    W_UV = np.ones((1, 1, 1))
+    hist = [(np.array([[1.0], [2.0]]), np.array([[0.0, 0.0, 1.0, 0.0], [0.0, 0.0, 1.0, 0.0]]))]
+    qn = np.zeros((1, 1, 1, 1))
+    qr = np.array([[[[0.0, 0.0, 1.0, 0.0]]]])
+    s0, s1 = math.cos(a) / math.sqrt(5.0), 1.0 / math.sqrt(5.0)
+    expect = (1.0 * math.exp(s0) + 2.0 * math.exp(s1)) / (math.exp(s0) + math.exp(s1))
+    out_e = decode_expanded(qn, qr, W_UK, W_UV, hist, q_len=1, base=base)
+    out_a = decode_absorbed(qn, qr, W_UK, W_UV, hist, q_len=1, base=base)
+    assert abs(out_e[0, 0, 0, 0] - expect) < 1e-14
+    assert abs(out_a[0, 0, 0, 0] - expect) < 1e-14
+    # the cached key rows written for those tokens carry the same rotation
+    rows = cache_rows(hist[0][0], hist[0][1], np.arange(2), base)
+    np.testing.assert_allclose(rows[1, 1:], [0.0, 0.0, math.cos(a), math.sin(a)], atol=1e-15)
+
+
+def test_scores_depend_on_relative_position_only_at_any_base():
+    # The RoPE score of a query at m and a key at n, at a non-default base, equals
+    # the closed form of turning each pair by (m - n) theta_k, theta_k = base**(-2k/d):
+    #   (q0 k0 + q1 k1) cos((m-n) theta_k) + (q0 k1 - q1 k0) sin((m-n) theta_k).
+    base = 777.0
+    rng = np.random.default_rng(14)
+    q, k = rng.standard_normal(8), rng.standard_normal(8)
+    for m, n in [(9, 4), (1000, 3)]:
+        lhs = rope(q, m, base) @ rope(k, n, base)
+        inv = base ** (-2.0 * np.arange(4) / 8.0)
+        ang = (m - n) * inv
+        # closed form of the pairwise rotation by (m - n) theta_k
+        rhs = sum((q[2 * i] * k[2 * i] + q[2 * i + 1] * k[2 * i + 1]) * math.cos(ang[i])
+                  + (q[2 * i] * k[2 * i + 1] - q[2 * i + 1] * k[2 * i]) * math.sin(ang[i]) for i in range(4))
+        assert abs(lhs - rhs) < 1e-9
+
+
 def test_hand_derived_causal_pair():
     # q_len = 2, T = 2, same one-dimensional set-up with q_R = 0: query 0 sits at
     # position 0 and sees key 0 only, so out = c_0 = 1; query 1 sees both keys.
