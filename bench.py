@@ -3,13 +3,15 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload v3_b1] [--impl ours|reference]
 
-A step is one pass of the whole hot path on one batch: append the q_len new
-tokens of every sequence to the compressed cache, then decode (absorb the
-query through W_UK, attend over the cache in latent space, combine split
-partials, project through W_UV).  The cache and the weights are resident in
-HBM; the timed region covers the device work of K steps (CUDA-graph replays,
-CUDA events on the launching stream), with L2 flushed by a 256 MiB write
-before every step, untimed.  One JSON line is printed by rank 0.
+The timed step is one mla_decode call on one batch: absorb the query through
+W_UK, attend over the compressed cache in latent space, merge split
+partials, project through W_UV.  The append of the step's q_len new tokens
+per sequence (mla_append_cache) is timed on its own and reported beside it.
+The cache and the weights are resident in HBM; the timed region covers the
+device work of K steps (CUDA-graph replays, CUDA events on the launching
+stream), with L2 flushed by a 256 MiB write before every step, untimed; a
+second pass without the flush gives the warm-L2 figure.  One JSON line is
+printed by rank 0.
 
 Multi-GPU (torchrun): every rank runs an independent replica of the workload
 on its own sequences (sequences are independent; nothing is exchanged on the
@@ -33,7 +35,7 @@ sys.path.insert(0, ROOT)
 
 from latent_compressed_attention_absorbed_b200 import workload as wl  # noqa: E402
 
-DEFAULT_WORKLOAD = "v3_b1"
+DEFAULT_WORKLOAD = "v3_ragged"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.json")
@@ -58,8 +60,8 @@ def work(cfg):
         "project": {"bytes": H * dv * dc * es + olat + U * H * dv * es, "flops": 2 * U * H * dc * dv},
         "append": {"bytes": 2 * U * (dc + dr) * es, "flops": 0},
     }
-    step = {
-        "bytes": cache + 2 * H * dn * dc * es + U * H * (dn + dr) * es + U * H * dv * es + 2 * U * (dc + dr) * es,
+    step = {  # one mla_decode call (the append is timed on its own)
+        "bytes": cache + 2 * H * dn * dc * es + U * H * (dn + dr) * es + U * H * dv * es,
         "flops": k["absorb"]["flops"] + k["attend"]["flops"] + k["project"]["flops"],
         "cache_bytes": cache,
     }
@@ -210,14 +212,17 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     assert lib.device_status() == 0
 
-    def step(stream=None, opts=None):
+    def append(stream=None):
         lib.append_cache(dims, cache, c_new, k_new, pos, stream=stream)
+
+    def step(stream=None, opts=None):
         lib.decode(dims, q_nope, q_rope, W_UK, W_UV, cache, seqlens, out=out, workspace=ws, opts=opts, stream=stream)
 
-    # ---- capture the step in a CUDA graph
+    # ---- capture the decode step, and the append on its own, in CUDA graphs
     s = torch.cuda.Stream(device)
     s.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(s):
+        append(stream=s)
         step(stream=s)
     torch.cuda.current_stream().wait_stream(s)
     status = lib.device_status()
@@ -231,6 +236,9 @@ def run_ours(args, rank, world, local_rank):
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=s):
         step(stream=s)
+    g_app = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_app, stream=s):
+        append(stream=s)
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
 
@@ -259,14 +267,35 @@ def run_ours(args, rank, world, local_rank):
             ends[i].record(stream)
         torch.cuda.synchronize()
     times_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
+
+    def timed_loop(graph, flush_between):
+        st = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        en = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        torch.cuda.synchronize()
+        for i in range(args.steps):
+            if flush_between:
+                busy()
+            st[i].record(stream)
+            graph.replay()
+            en[i].record(stream)
+        torch.cuda.synchronize()
+        return float(np.mean([a.elapsed_time(b) for a, b in zip(st, en)]))
+
+    # ---- the same decode with L2 warm (no flush between replays), and the append alone (flushed)
+    for _ in range(3):
+        g.replay()
+    ms_warm = timed_loop(g, flush_between=False)
+    for _ in range(3):
+        g_app.replay()
+    ms_append = timed_loop(g_app, flush_between=True)
     if world > 1:
         torch.distributed.barrier()
     ms_step = float(np.mean(times_ms))
     ms_med = float(np.median(times_ms))
     if world > 1:
-        t = torch.tensor([ms_step, ms_med], dtype=torch.float64, device=device)
+        t = torch.tensor([ms_step, ms_med, ms_warm, ms_append], dtype=torch.float64, device=device)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_step, ms_med = float(t[0]), float(t[1])
+        ms_step, ms_med, ms_warm, ms_append = (float(x) for x in t)
 
     # ---- per-kernel stage times (same kernels, launched directly with stage events)
     n_ev = binding.NUM_EVENTS
@@ -289,18 +318,14 @@ def run_ours(args, rank, world, local_rank):
     e2e = None
     if not args.no_e2e:
         pin = lambda st: torch.from_numpy(st.raw.view(np.int16) if st.dtype == "bf16" else st.raw).pin_memory()
-        h_qn, h_qr, h_c, h_k = pin(qn_h), pin(qr_h), pin(c_new_h), pin(k_new_h)
+        h_qn, h_qr = pin(qn_h), pin(qr_h)
         h_out = torch.empty(out.shape, dtype=torch.int16 if cfg.dtype == "bf16" else torch.float32).pin_memory()
         d_qn, d_qr = torch.empty_like(h_qn, device=device), torch.empty_like(h_qr, device=device)
-        d_c, d_k = torch.empty_like(h_c, device=device), torch.empty_like(h_k, device=device)
         view = (lambda t: t.view(torch.bfloat16)) if cfg.dtype == "bf16" else (lambda t: t)
 
         def e2e_step():
             d_qn.copy_(h_qn, non_blocking=True)
             d_qr.copy_(h_qr, non_blocking=True)
-            d_c.copy_(h_c, non_blocking=True)
-            d_k.copy_(h_k, non_blocking=True)
-            lib.append_cache(dims, cache, view(d_c), view(d_k), pos)
             o = lib.decode(dims, view(d_qn), view(d_qr), W_UK, W_UV, cache, seqlens, out=out, workspace=ws)
             h_out.copy_(o.view(torch.int16) if cfg.dtype == "bf16" else o, non_blocking=True)
             torch.cuda.current_stream().synchronize()
@@ -319,11 +344,12 @@ def run_ours(args, rank, world, local_rank):
             t = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
             torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
             e2e_ms = float(t[0])
-        h2d = sum(x.numel() * x.element_size() for x in (h_qn, h_qr, h_c, h_k))
+        h2d = sum(x.numel() * x.element_size() for x in (h_qn, h_qr))
         d2h = h_out.numel() * h_out.element_size()
         e2e = {"value": round(e2e_ms * 1e3, 3), "unit": "us/step", "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h), "timing": "host wall clock per step incl. synchronize"}
-    return cfg, path, ms_step, ms_med, stage_ms, clk.summary(), e2e
+    times = {"ms_step": ms_step, "ms_med": ms_med, "ms_warm": ms_warm, "ms_append": ms_append}
+    return cfg, path, times, stage_ms, clk.summary(), e2e
 
 
 class OracleSample:
@@ -396,8 +422,8 @@ def config_of(cfg, args):
                         f"q_len={cfg.q_len}, H={cfg.H}, d_c={cfg.d_c}, d_r={cfg.d_r}, d_n={cfg.d_n}, d_v={cfg.d_v}, "
                         f"{cfg.dtype}",
             "B": cfg.B, "seq_len": int(max(cfg.seqlens)), "sum_seqlens": int(sum(cfg.seqlens)), "q_len": cfg.q_len,
-            "step": "append q_len tokens/sequence + decode (absorb, attend, combine, W_UV)",
-            "l2": "flushed before every step (256 MiB write, untimed)",
+            "step": "one mla_decode call (absorb, attend, combine, W_UV); the q_len-token append is timed apart",
+            "l2": "flushed before every step (256 MiB write, untimed); warm_l2_us_per_step without the flush",
             "parallelism": f"replicas x{args.gpus} (sequences are independent; no collective on the data path)"}
 
 
@@ -430,7 +456,8 @@ def main():
         torch.cuda.set_device(local_rank)
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local_rank))
-    cfg, path, ms_step, ms_med, stage_ms, clocks, e2e = run_ours(args, rank, world, local_rank)
+    cfg, path, times, stage_ms, clocks, e2e = run_ours(args, rank, world, local_rank)
+    ms_step, ms_med = times["ms_step"], times["ms_med"]
     if world > 1:
         import torch
         torch.distributed.barrier()
@@ -455,6 +482,11 @@ def main():
              "attend": "mla_attend_kernel",
              "project": "project_gemv_kernel" if rows <= 8 else "head_gemm_kernel (W_UV project)"}[dom]
     traffic = traffic_for(cfg.name, kname)
+    # The library prefetches W_UV into L2 from inside the attention kernel when
+    # the cache read is small (at most 64 MiB over B x T_max rows), for the
+    # projection that follows; those bytes are the projection's, not attention's.
+    prefetch = (cfg.H * cfg.d_v * cfg.d_c * 2 if dom == "attend" and
+                cfg.B * cfg.T_max * cfg.row * 2 <= (64 << 20) else 0)
     roof = {"kernel": kname, "bound": "hbm" if hbm_bound else "tensor",
             "achieved": round((kb / kt / 1e9) if hbm_bound else (kf / kt / 1e12), 2),
             "peak": pk["hbm_gbs"] if hbm_bound else pk["bf16_tflops"],
@@ -462,6 +494,7 @@ def main():
             "traffic": traffic,
             "algorithmic_bytes": int(kb), "algorithmic_flops": int(kf),
             "kernel_us": round(kt * 1e6, 3),
+            "l2_prefetch_bytes_in_traffic": int(prefetch),
             "peak_source": f"{pk_kind} (MEASURED_PEAKS.json burst figure)" if pk_kind == "measured" else "fallback"}
     roof["frac"] = round(roof["achieved"] / roof["peak"], 4)
     t_step = ms_step * 1e-3
@@ -487,10 +520,13 @@ def main():
         "tflops": round(step_work["flops"] / t_step / 1e12, 2),
         "step_roofline_us": round(step_roof_s * 1e6, 3),
         "step_roofline_frac": round(step_roof_s / t_step, 4),
+        "warm_l2_us_per_step": round(times["ms_warm"] * 1e3, 3),
+        "append_us": round(times["ms_append"] * 1e3, 3),
+        "step_with_append_us": round((ms_step + times["ms_append"]) * 1e3, 3),
         "stage_us": {k: round(v * 1e3, 3) for k, v in stage_ms.items()},
         "roofline": roof,
-        # append + absorb + attend (+ combine above 8 query rows) + project per step
-        "gpu_launches": ((4 if rows <= 8 else 5) if path == "sm100" else 4) * args.steps * args.gpus,
+        # absorb + attend (+ combine above 8 query rows) + project per timed step
+        "gpu_launches": ((3 if rows <= 8 else 4) if path == "sm100" else 3) * args.steps * args.gpus,
         "clocks": clocks,
         "e2e": e2e,
     }

@@ -52,6 +52,11 @@ class MLAConfig:
     w_std: float
     seed: int
     rope_base: float = 10000.0
+    # 0: W_UK ~ N(0, w_std).  Otherwise W_UK[h][d][c] = w_uk_select when
+    # d == c % d_n and 0 elsewhere: every folded query component is then a
+    # query component times w_uk_select, exactly representable in the storage
+    # dtype when w_uk_select is a power of two (sharp-score test inputs).
+    w_uk_select: float = 0.0
 
     @property
     def T_max(self) -> int:
@@ -130,7 +135,13 @@ def _normal(seed: int, tag: int, index: int, shape, std: float = 1.0) -> np.ndar
 
 def weights(cfg: MLAConfig):
     """W_UK, W_UV as [H, d_n, d_c] and [H, d_v, d_c] (k_C = W_UK[h] @ c, v = W_UV[h] @ c)."""
-    w_uk = Stored(_normal(cfg.seed, _TAG_W_UK, 0, (cfg.H, cfg.d_n, cfg.d_c), cfg.w_std), cfg.dtype)
+    if cfg.w_uk_select:
+        sel = np.zeros((cfg.H, cfg.d_n, cfg.d_c))
+        c = np.arange(cfg.d_c)
+        sel[:, c % cfg.d_n, c] = cfg.w_uk_select
+        w_uk = Stored(sel, cfg.dtype)
+    else:
+        w_uk = Stored(_normal(cfg.seed, _TAG_W_UK, 0, (cfg.H, cfg.d_n, cfg.d_c), cfg.w_std), cfg.dtype)
     w_uv = Stored(_normal(cfg.seed, _TAG_W_UV, 0, (cfg.H, cfg.d_v, cfg.d_c), cfg.w_std), cfg.dtype)
     return w_uk, w_uv
 

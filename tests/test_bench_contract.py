@@ -26,7 +26,7 @@ def test_reference_arm_prints_one_contract_line():
     assert d["impl"] == "reference"
     assert d["unit"] == "us/step" and d["higher_is_better"] is False
     assert d["value"] > 0 and d["steps"] == 1 and d["warmup"] >= 3
-    assert d["config"]["workload"].startswith("v3_b1")
+    assert d["config"]["workload"].startswith("v3_ragged")
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": "us/step", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}

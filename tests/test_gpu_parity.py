@@ -8,7 +8,7 @@ import numpy as np
 import pytest
 import torch
 
-from oracle import cache_rows
+from oracle import cache_rows, decode_absorbed, decode_expanded
 from latent_compressed_attention_absorbed_b200 import workload as wl
 from mla_testutil import Problem, as_f64, check_close, dims_of, to_device, torch_dtype
 
@@ -146,6 +146,43 @@ def test_bad_seqlens_are_flagged_and_zeroed(lib):
     check_close(as_f64(out[:1]), P.oracle_expanded([0])[:1], "bf16", "valid sequence")
 
 
+# Sharp softmax.  W_UK = 8 x a selection matrix makes every folded query
+# component a query component times 8, exactly representable in bf16, so the
+# folded query carries no rounding and the score error comes only from the
+# kernel's own score arithmetic (the pair's exchange of partial scores).
+# Scores then span about +-80 log2 units (std ~19), and the softmax still
+# spreads its weight over several keys.  (Scaling a random query instead
+# mostly measures the bf16 rounding of the folded query, which grows with the
+# scores and is inherent to a bf16 absorbed path.)
+SHARP_CASES = [
+    ((4096,), 1, 0),
+    ((3000, 700), 2, 8),      # split pieces, causal pair
+    ((4096, 5, 64), 1, 40),   # many pieces merged by the projection kernel
+    ((2000,) * 9, 1, 3),      # more than eight query rows: tensor-core GEMMs and the combine kernel
+]
+
+
+@pytest.mark.parametrize("seqlens,q_len,pairs", SHARP_CASES)
+def test_sharp_scores_against_expanded_oracle(lib, seqlens, q_len, pairs):
+    cfg = _v3(seqlens, q_len, seed=13).with_(w_uk_select=8.0)
+    P = Problem(lib, cfg)
+    out = P.decode(opts=lib.opts(num_pairs=pairs))
+    assert lib.last_path() == "sm100"
+    assert lib.device_status() == 0
+    check_close(as_f64(out), P.oracle_expanded(range(cfg.B)), "bf16", f"sharp {seqlens} q_len={q_len}")
+
+
+@pytest.mark.parametrize("base", [500.0, 1.0e6])
+def test_rope_base_through_append_and_decode(lib, base):
+    # The cache append rotates k_R and the absorb step rotates q_R with the
+    # caller's base; the oracle rotates both with the same base.
+    cfg = _v3((700, 333, 65), 2, seed=17).with_(rope_base=base)
+    P = Problem(lib, cfg)
+    out = P.decode(opts=lib.opts(num_pairs=4))
+    assert lib.last_path() == "sm100"
+    check_close(as_f64(out), P.oracle_expanded(range(cfg.B)), "bf16", f"rope_base={base}")
+
+
 def test_repeat_runs_are_bitwise_equal(lib):
     cfg = _v3((900, 77), 2)
     P = Problem(lib, cfg)
@@ -201,8 +238,26 @@ def test_workload_v3_b64_sampled(lib):
     _sampled(lib, "v3_b64", [0, 31, 63], [0, 77, 127])
 
 
-def test_workload_v3_long_sampled(lib):
-    _sampled(lib, "v3_long", [0, 5], [3, 64])
+def test_workload_v3_long_every_sequence(lib):
+    # All 8 sequences of 128K tokens: every head through the fp64 absorbed form
+    # and 4 heads (one per TMEM lane quarter) through the fp64 expanded
+    # definition.  Histories are regenerated one sequence at a time.
+    cfg = wl.CONFIGS["v3_long"]
+    P = Problem(lib, cfg, keep_history=[])
+    out = as_f64(P.decode())
+    assert lib.last_path() == "sm100"
+    assert lib.device_status() == 0
+    assert np.all(np.isfinite(out))
+    heads = [0, 37, 70, 127]
+    for b in range(cfg.B):
+        c, k = wl.sequence_history(cfg, b)
+        hist = [(None, None)] * cfg.B
+        hist[b] = (c.values, k.values)
+        del c, k
+        args = (P.q_nope.values, P.q_rope.values, P.w_uk.values, P.w_uv.values, hist, cfg.q_len, cfg.rope_base)
+        check_close(out[b], decode_absorbed(*args, seqs=[b])[b], "bf16", f"v3_long seq {b} absorbed-oracle")
+        ref = decode_expanded(*args, seqs=[b], heads=heads)[b]
+        check_close(out[b][:, heads], ref[:, heads], "bf16", f"v3_long seq {b} expanded-oracle")
 
 
 def test_workload_v3_ragged_sampled(lib):
