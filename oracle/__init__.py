@@ -2,7 +2,9 @@
 from .mla_oracle import (  # noqa: F401
     cache_elements_per_token,
     cache_rows,
+    cache_rows_from_hidden,
     decode_absorbed,
     decode_expanded,
+    rms_norm,
     rope,
 )

@@ -65,7 +65,9 @@ import numpy as np
 
 __all__ = [
     "rope",
+    "rms_norm",
     "cache_rows",
+    "cache_rows_from_hidden",
     "decode_expanded",
     "decode_absorbed",
     "cache_elements_per_token",
@@ -103,6 +105,35 @@ def cache_rows(c_kv: np.ndarray, k_rope: np.ndarray, positions, base: float = 10
     """
     c_kv = np.asarray(c_kv, dtype=np.float64)
     return np.concatenate([c_kv, rope(k_rope, positions, base)], axis=-1)
+
+
+def rms_norm(v: np.ndarray, gamma: np.ndarray, eps: float = 1e-6) -> np.ndarray:
+    """RMSNorm over the last axis: v / sqrt(mean(v^2) + eps) * gamma.
+
+    [P5] section 1 names RMSNorm as the normalisation of the V3 block
+    (Pre-Norm), and its configuration block gives rms_norm_eps = 1e-6.
+    """
+    v = np.asarray(v, dtype=np.float64)
+    return v / np.sqrt(np.mean(v * v, axis=-1, keepdims=True) + eps) * np.asarray(gamma, dtype=np.float64)
+
+
+def cache_rows_from_hidden(x: np.ndarray, W_DKV: np.ndarray, W_KR: np.ndarray, gamma: np.ndarray, positions,
+                           base: float = 10000.0, eps: float = 1e-6) -> np.ndarray:
+    """Cache rows computed from the attention block's input x (hidden size d):
+    [ RMSNorm_gamma(W_DKV x) || RoPE(W_KR x, position) ].
+
+    [P5] section 2.2 and [P1] section 二: the latent is a down-projection of
+    the hidden state, c^KV = W^DKV h (d_c = 512 of hidden 7168); [P3]'s MLA
+    panel: the hidden state is projected to c_KV and to the decoupled RoPE key
+    k_R, which is stored rotated.  The RMSNorm of the latent (gain gamma) is
+    the reading that gives the cached latent its unit scale; x is the block's
+    input after its own pre-norm.
+    x [..., d]; W_DKV [d_c, d]; W_KR [d_r, d]; gamma [d_c]; positions broadcast to x.shape[:-1].
+    """
+    x = np.asarray(x, dtype=np.float64)
+    c = x @ np.asarray(W_DKV, dtype=np.float64).T
+    k = x @ np.asarray(W_KR, dtype=np.float64).T
+    return np.concatenate([rms_norm(c, gamma, eps), rope(k, positions, base)], axis=-1)
 
 
 def _softmax(s: np.ndarray) -> np.ndarray:

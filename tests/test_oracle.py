@@ -11,7 +11,8 @@ import os
 import numpy as np
 import pytest
 
-from oracle import cache_elements_per_token, cache_rows, decode_absorbed, decode_expanded, rope
+from oracle import (cache_elements_per_token, cache_rows, cache_rows_from_hidden, decode_absorbed, decode_expanded,
+                    rms_norm, rope)
 from latent_compressed_attention_absorbed_b200 import workload as wl
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
@@ -93,6 +94,52 @@ def test_cache_rows_layout():
     np.testing.assert_array_equal(rows[:, :10], c)
     np.testing.assert_array_equal(rows[0, 10:], k[0])
     np.testing.assert_allclose(rows[2, 10:], rope(k[2], 9), atol=1e-15)
+
+
+# ------------------------------------------------------------------ cache rows from the hidden state
+
+def test_rms_norm_hand_example_and_invariants():
+    # v = (3, 4): mean of squares 12.5, so v / sqrt(12.5 + eps) * gamma.
+    eps = 1e-6
+    got = rms_norm(np.array([3.0, 4.0]), np.array([2.0, -1.0]), eps)
+    d = math.sqrt(12.5 + eps)
+    np.testing.assert_allclose(got, [6.0 / d, -4.0 / d], rtol=1e-15)
+    rng = np.random.default_rng(15)
+    v = rng.standard_normal((5, 512))
+    # scale invariance (eps = 0) and unit rms with gamma = 1
+    np.testing.assert_allclose(rms_norm(v * 37.0, np.ones(512), 0.0), rms_norm(v, np.ones(512), 0.0), rtol=1e-13)
+    np.testing.assert_allclose(np.sqrt(np.mean(rms_norm(v, np.ones(512), 0.0) ** 2, axis=-1)), 1.0, rtol=1e-13)
+
+
+def test_cache_rows_from_hidden_hand_example():
+    # d = 2, d_c = 2, d_r = 2: x = (1, 2); W_DKV = I -> c = (1, 2), mean square 2.5;
+    # W_KR = [[1, 1], [0, 1]] -> k = (3, 2), rotated at position p by angle p (pair 0).
+    x = np.array([[1.0, 2.0]])
+    W_DKV = np.eye(2)
+    W_KR = np.array([[1.0, 1.0], [0.0, 1.0]])
+    gamma = np.array([0.5, 3.0])
+    p, eps = 5, 1e-6
+    rows = cache_rows_from_hidden(x, W_DKV, W_KR, gamma, np.array([p]), eps=eps)
+    d = math.sqrt(2.5 + eps)
+    np.testing.assert_allclose(rows[0], [0.5 / d, 6.0 / d, 3 * math.cos(p) - 2 * math.sin(p),
+                                         3 * math.sin(p) + 2 * math.cos(p)], rtol=1e-14, atol=1e-15)
+
+
+def test_cache_rows_from_hidden_properties():
+    rng = np.random.default_rng(16)
+    x = rng.standard_normal((3, 40))
+    W_DKV, W_KR = rng.standard_normal((12, 40)), rng.standard_normal((4, 40))
+    gamma = rng.standard_normal(12)
+    pos = np.array([0, 7, 300])
+    rows = cache_rows_from_hidden(x, W_DKV, W_KR, gamma, pos, eps=0.0)
+    # the latent part does not change when x is scaled (RMSNorm after a linear map)
+    rows2 = cache_rows_from_hidden(4.5 * x, W_DKV, W_KR, gamma, pos, eps=0.0)
+    np.testing.assert_allclose(rows2[:, :12], rows[:, :12], rtol=1e-12)
+    # the RoPE part is linear in x and keeps the norm of W_KR x
+    np.testing.assert_allclose(rows2[:, 12:], 4.5 * rows[:, 12:], rtol=1e-12)
+    np.testing.assert_allclose(np.linalg.norm(rows[:, 12:], axis=1), np.linalg.norm(x @ W_KR.T, axis=1), rtol=1e-12)
+    # position 0 leaves the key unrotated
+    np.testing.assert_allclose(rows[0, 12:], W_KR @ x[0], rtol=1e-12)
 
 
 # ------------------------------------------------------------------ decode: closed forms
