@@ -35,6 +35,7 @@ import numpy as np
 
 # Stream tags: one per tensor kind.
 _TAG_W_UK, _TAG_W_UV, _TAG_Q_NOPE, _TAG_Q_ROPE, _TAG_C_KV, _TAG_K_ROPE, _TAG_NEW = range(7)
+_TAG_X, _TAG_W_A, _TAG_GAMMA, _TAG_W_O = range(7, 11)
 
 
 @dataclasses.dataclass(frozen=True)
@@ -57,6 +58,7 @@ class MLAConfig:
     # query component times w_uk_select, exactly representable in the storage
     # dtype when w_uk_select is a power of two (sharp-score test inputs).
     w_uk_select: float = 0.0
+    d_model: int = 7168  # hidden size of the block (the projections around the decode)
 
     @property
     def T_max(self) -> int:
@@ -170,6 +172,24 @@ def new_tokens(cfg: MLAConfig, n_tok: int, index: int = 0):
     c = Stored(_normal(cfg.seed, _TAG_NEW, 2 * index, (cfg.B, n_tok, cfg.d_c)), cfg.dtype)
     k = Stored(_normal(cfg.seed, _TAG_NEW, 2 * index + 1, (cfg.B, n_tok, cfg.d_r)), cfg.dtype)
     return c, k
+
+
+def block_input(cfg: MLAConfig, n_tok: int, index: int = 0):
+    """The attention block's input x [B, n_tok, d_model] ~ N(0, 1) (unit rms, as after the block's pre-norm)."""
+    return Stored(_normal(cfg.seed, _TAG_X, index, (cfg.B, n_tok, cfg.d_model)), cfg.dtype)
+
+
+def append_weights(cfg: MLAConfig):
+    """W_A = [W_DKV; W_KR] as [d_c + d_r, d_model] ~ N(0, w_std), and the latent's RMSNorm gain
+    gamma [d_c] ~ N(1, 0.1)."""
+    w_a = Stored(_normal(cfg.seed, _TAG_W_A, 0, (cfg.d_c + cfg.d_r, cfg.d_model), cfg.w_std), cfg.dtype)
+    gamma = Stored(1.0 + _normal(cfg.seed, _TAG_GAMMA, 0, (cfg.d_c,), 0.1), cfg.dtype)
+    return w_a, gamma
+
+
+def output_weights(cfg: MLAConfig):
+    """W_O [d_model, H * d_v] ~ N(0, w_std)."""
+    return Stored(_normal(cfg.seed, _TAG_W_O, 0, (cfg.d_model, cfg.H * cfg.d_v), cfg.w_std), cfg.dtype)
 
 
 def small_variant(cfg: MLAConfig, B: Optional[int] = None, seqlens: Optional[Sequence[int]] = None,

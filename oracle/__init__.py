@@ -5,6 +5,7 @@ from .mla_oracle import (  # noqa: F401
     cache_rows_from_hidden,
     decode_absorbed,
     decode_expanded,
+    output_projection,
     rms_norm,
     rope,
 )

@@ -71,6 +71,7 @@ __all__ = [
     "decode_expanded",
     "decode_absorbed",
     "cache_elements_per_token",
+    "output_projection",
 ]
 
 
@@ -221,6 +222,19 @@ def decode_absorbed(q_nope: np.ndarray, q_rope: np.ndarray, W_UK: np.ndarray, W_
             olat[b, i] = o
             out[b, i] = np.einsum("hvc,hc->hv", W_UV, o)
     return (out, olat) if return_latent else out
+
+
+def output_projection(out: np.ndarray, W_O: np.ndarray) -> np.ndarray:
+    """The block's output projection after W_UV: y = W_O concat_h(out_h).
+
+    [P3]'s MLA panel: aggregate sum_j p_j c_KV,j, then W_UV and the output
+    projection; the MLA steps of the taojin168.com forum page (section 2.1,
+    last step): the attention output is mapped back to the model width.
+    out [..., H, d_v]; W_O [d, H * d_v] (head-major columns).  Returns [..., d].
+    """
+    out = np.asarray(out, dtype=np.float64)
+    flat = out.reshape(out.shape[:-2] + (out.shape[-2] * out.shape[-1],))
+    return flat @ np.asarray(W_O, dtype=np.float64).T
 
 
 def cache_elements_per_token(H: int, d_c: int, d_r: int, d_n: int, d_v: int):

@@ -12,7 +12,7 @@ import numpy as np
 import pytest
 
 from oracle import (cache_elements_per_token, cache_rows, cache_rows_from_hidden, decode_absorbed, decode_expanded,
-                    rms_norm, rope)
+                    output_projection, rms_norm, rope)
 from latent_compressed_attention_absorbed_b200 import workload as wl
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
@@ -140,6 +140,26 @@ def test_cache_rows_from_hidden_properties():
     np.testing.assert_allclose(np.linalg.norm(rows[:, 12:], axis=1), np.linalg.norm(x @ W_KR.T, axis=1), rtol=1e-12)
     # position 0 leaves the key unrotated
     np.testing.assert_allclose(rows[0, 12:], W_KR @ x[0], rtol=1e-12)
+
+
+def test_output_projection_hand_example():
+    # H = 2, d_v = 2, d = 1: out = [[1, 2], [3, 4]] (head-major) and W_O = [[10, 20, 30, 40]]
+    # give y = 10 + 40 + 90 + 160 = 300.
+    y = output_projection(np.array([[1.0, 2.0], [3.0, 4.0]]), np.array([[10.0, 20.0, 30.0, 40.0]]))
+    assert y.shape == (1,) and y[0] == 300.0
+
+
+def test_output_projection_folds_with_W_UV():
+    # W_O (W_UV o) = (W_O W_UV) o per head: projecting the decode's per-head
+    # outputs equals applying the folded per-head maps W_O[:, h] W_UV[h] to the
+    # latent aggregates o_h (associativity; the order the pages describe).
+    rng = np.random.default_rng(17)
+    qn, qr, W_UK, W_UV, hist = _rand_problem(rng)
+    W_O = rng.standard_normal((7, 3 * 5))
+    out, olat = decode_absorbed(qn, qr, W_UK, W_UV, hist, q_len=1, return_latent=True)
+    y = output_projection(out, W_O)
+    folded = sum(olat[..., h, :] @ (W_O[:, 5 * h:5 * h + 5] @ W_UV[h]).T for h in range(3))
+    np.testing.assert_allclose(y, folded, rtol=1e-12)
 
 
 # ------------------------------------------------------------------ decode: closed forms
