@@ -143,6 +143,14 @@ int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_rope,
  *         n_events >= MLA_NUM_EVENTS, mla_decode_ex records them on `stream`
  *         at the stage boundaries listed below, so a caller can time each
  *         kernel with cudaEventElapsedTime.  The library does not own them.
+ *   wait_limit_ns: time limit of each device-side barrier wait of the
+ *         attention kernel (0 = default, 2 s).  A wait that runs out sets
+ *         MLA_STATUS_TIMEOUT; the kernel then stops, drains what it has in
+ *         flight and exits, leaving the context usable.
+ *   withhold_tile: test hook for that path; 0 = off.  A value k > 0 makes
+ *         the attention kernel's loader stop before the k-th 64-key tile of
+ *         each cluster, so a bounded wait runs out and the call reports
+ *         MLA_STATUS_TIMEOUT (the result is then undefined).
  *   All-zero options are valid (overhead_tiles 0 charges nothing per sequence). */
 typedef struct {
     int32_t path;
@@ -151,6 +159,9 @@ typedef struct {
     int32_t min_tiles;
     int32_t n_events;
     void* const* events;
+    int64_t wait_limit_ns;
+    int32_t withhold_tile;
+    int32_t reserved;
 } mla_decode_opts_t;
 
 /* Event slots recorded by mla_decode_ex (sm_100a path; the generic path
@@ -219,6 +230,48 @@ int mla_attend_latent(const mla_dims_t* dims, const void* q_hat, const mla_cache
 int mla_project_out(const mla_dims_t* dims, const void* o_lat, const void* W_UV,
                     int32_t rows, void* out, const mla_decode_opts_t* opts,
                     mla_stream_t stream);
+
+/* ---------------------------------------------------------------- projections around the decode
+ * Both are dense bf16 contractions on the tensor cores (split over K so that
+ * a few hundred tokens still spread the weight read over every SM); both
+ * need bf16, the V3 head geometry (d_c 512, d_r 64, H 128, d_v 128) and a
+ * compute-capability 10.0 device (MLA_ERR_UNSUPPORTED otherwise), and
+ * d_model a multiple of 64.  Each takes a workspace (fp32 split partials)
+ * of the size its *_workspace_bytes() returns, 16-byte aligned, owned by
+ * the call until the stream reaches its end.
+ *
+ * Cache append from the attention block's input (a1 with the projections
+ * that produce its inputs fused in):
+ *   row pos[b]+i of sequence b = [ RMSNorm_gamma(W_DKV x[b][i]) || RoPE(W_KR x[b][i], pos[b]+i) ]
+ * (m.lsln.cn/news/222502 section 2.2: c^KV = W^DKV h; section 1: RMSNorm,
+ *  rms_norm_eps 1e-6 in its configuration block; 092 page, section 二: the
+ *  cache keeps the latent and the decoupled RoPE key;
+ *  ailearn.mscapital.top MLA panel: the hidden state is projected to c_KV
+ *  and k_R).  The RMSNorm is taken over the d_c latent values in fp32.
+ *   x      [B][n_tok][d_model]   block input (after the block's own pre-norm)
+ *   W_A    [d_c + d_r][d_model]  rows 0..d_c-1 hold W_DKV, rows d_c.. hold W_KR
+ *   gamma  [d_c]                 RMSNorm gain of the latent
+ *   pos    [B] int32             position of the first new token of sequence b
+ * Rows with an out-of-range position are skipped and set MLA_STATUS_BAD_POS. */
+size_t mla_append_from_hidden_workspace_bytes(const mla_dims_t* dims, int32_t B, int32_t n_tok, int32_t d_model);
+int mla_append_from_hidden(const mla_dims_t* dims, const void* x, const void* W_A, const void* gamma,
+                           const int32_t* pos, int32_t B, int32_t n_tok, int32_t d_model,
+                           const mla_cache_t* cache, void* workspace, size_t workspace_bytes,
+                           mla_stream_t stream);
+
+/* Output projection of the attention block: y[r] = W_O out[r], where out[r]
+ * is a decode output row viewed as H * d_v values (head-major)
+ * (ailearn.mscapital.top MLA panel: aggregate in latent space, then W_UV and
+ * the output projection; taojin168.com forum page, section 2.1, the MLA
+ * steps' last step: an output projection maps the attention output back to
+ * the model width).
+ *   attn_out [rows][H * d_v]     e.g. mla_decode's out, [B * q_len][H][d_v]
+ *   W_O      [d_model][H * d_v]
+ *   y        [rows][d_model]     written */
+size_t mla_output_projection_workspace_bytes(const mla_dims_t* dims, int32_t rows, int32_t d_model);
+int mla_output_projection(const mla_dims_t* dims, const void* attn_out, const void* W_O, int32_t rows,
+                          int32_t d_model, void* y, void* workspace, size_t workspace_bytes,
+                          mla_stream_t stream);
 
 /* ---------------------------------------------------------------- status */
 

@@ -29,7 +29,8 @@ ERRORS = {-1: "MLA_ERR_ARG", -2: "MLA_ERR_SHAPE", -3: "MLA_ERR_ALIGN", -4: "MLA_
 # Every symbol the header declares (checked by the CPU test suite).
 EXPORTS = ["mla_append_cache", "mla_workspace_bytes", "mla_decode", "mla_decode_ex", "mla_absorb_query",
            "mla_attend_latent", "mla_project_out", "mla_device_status", "mla_last_error", "mla_last_path",
-           "mla_version", "mla_decode_no_alloc"]
+           "mla_version", "mla_decode_no_alloc", "mla_append_from_hidden", "mla_append_from_hidden_workspace_bytes",
+           "mla_output_projection", "mla_output_projection_workspace_bytes"]
 
 
 class Dims(ctypes.Structure):
@@ -46,7 +47,8 @@ class Cache(ctypes.Structure):
 class Opts(ctypes.Structure):
     _fields_ = [("path", ctypes.c_int32), ("num_pairs", ctypes.c_int32), ("overhead_tiles", ctypes.c_int32),
                 ("min_tiles", ctypes.c_int32), ("n_events", ctypes.c_int32),
-                ("events", ctypes.POINTER(ctypes.c_void_p))]
+                ("events", ctypes.POINTER(ctypes.c_void_p)), ("wait_limit_ns", ctypes.c_int64),
+                ("withhold_tile", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 
 class MLAError(RuntimeError):
@@ -70,6 +72,11 @@ _SIGS = {
     "mla_attend_latent": ([ctypes.POINTER(Dims), _P, ctypes.POINTER(Cache), _P, _I, _I, _P, _P, ctypes.c_size_t,
                            ctypes.POINTER(Opts), _P], ctypes.c_int),
     "mla_project_out": ([ctypes.POINTER(Dims), _P, _P, _I, _P, ctypes.POINTER(Opts), _P], ctypes.c_int),
+    "mla_append_from_hidden_workspace_bytes": ([ctypes.POINTER(Dims), _I, _I, _I], ctypes.c_size_t),
+    "mla_append_from_hidden": ([ctypes.POINTER(Dims), _P, _P, _P, _P, _I, _I, _I, ctypes.POINTER(Cache), _P,
+                                ctypes.c_size_t, _P], ctypes.c_int),
+    "mla_output_projection_workspace_bytes": ([ctypes.POINTER(Dims), _I, _I], ctypes.c_size_t),
+    "mla_output_projection": ([ctypes.POINTER(Dims), _P, _P, _I, _I, _P, _P, ctypes.c_size_t, _P], ctypes.c_int),
     "mla_device_status": ([_P, ctypes.POINTER(_I)], ctypes.c_int),
     "mla_last_error": ([], ctypes.c_char_p),
     "mla_last_path": ([], ctypes.c_char_p),
@@ -134,9 +141,11 @@ class Library:
         return Cache(cache.data_ptr(), cache.shape[0], cache.shape[1], cache.stride(0), cache.stride(1))
 
     @staticmethod
-    def opts(path=PATH_AUTO, num_pairs=0, overhead_tiles=-1, min_tiles=0, events=None) -> Opts:
-        """``events``: MLA_NUM_EVENTS recorded torch.cuda.Event objects (stage timing)."""
-        o = Opts(path, num_pairs, overhead_tiles, min_tiles, 0, None)
+    def opts(path=PATH_AUTO, num_pairs=0, overhead_tiles=-1, min_tiles=0, events=None, wait_limit_ns=0,
+             withhold_tile=0) -> Opts:
+        """``events``: MLA_NUM_EVENTS recorded torch.cuda.Event objects (stage timing).
+        ``wait_limit_ns`` / ``withhold_tile``: see mla_decode_opts_t (the latter is a test hook)."""
+        o = Opts(path, num_pairs, overhead_tiles, min_tiles, 0, None, wait_limit_ns, withhold_tile, 0)
         if events is not None:
             arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
             o.events = ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p))
@@ -230,6 +239,39 @@ class Library:
         self._check(self.lib.mla_project_out(ctypes.byref(dims), _ptr(o_lat), _ptr(W_UV), rows, _ptr(out),
                                              ctypes.byref(o), _stream(stream)))
         return out
+
+    def append_from_hidden(self, dims: Dims, cache: torch.Tensor, x: torch.Tensor, W_A: torch.Tensor,
+                           gamma: torch.Tensor, pos: torch.Tensor, workspace=None, stream=None):
+        """Rows pos[b]+i of cache[b] <- [RMSNorm_gamma(W_DKV x[b,i]) || RoPE(W_KR x[b,i], pos[b]+i)];
+        W_A = [W_DKV; W_KR] as [d_c + d_r, d_model]."""
+        _need(x, "x", ndim=3)
+        _need(W_A, "W_A", ndim=2)
+        _need(gamma, "gamma", ndim=1)
+        _need(pos, "pos", dtype=torch.int32, ndim=1)
+        B, n_tok, d_model = x.shape
+        if workspace is None:
+            n = self.lib.mla_append_from_hidden_workspace_bytes(ctypes.byref(dims), B, n_tok, d_model)
+            workspace = torch.empty(max(int(n), 16), dtype=torch.uint8, device=x.device)
+        cd = self.cache_desc(cache)
+        self._check(self.lib.mla_append_from_hidden(ctypes.byref(dims), _ptr(x), _ptr(W_A), _ptr(gamma), _ptr(pos),
+                                                    B, n_tok, d_model, ctypes.byref(cd), _ptr(workspace),
+                                                    workspace.numel(), _stream(stream)))
+
+    def output_projection(self, dims: Dims, attn_out: torch.Tensor, W_O: torch.Tensor, y=None, workspace=None,
+                          stream=None):
+        """y[r] = W_O attn_out[r] with attn_out viewed as [rows, H * d_v]; W_O is [d_model, H * d_v]."""
+        _need(attn_out, "attn_out")
+        _need(W_O, "W_O", ndim=2)
+        width = dims.H * dims.d_v
+        rows, d_model = attn_out.numel() // width, W_O.shape[0]
+        if y is None:
+            y = torch.empty((rows, d_model), dtype=attn_out.dtype, device=attn_out.device)
+        if workspace is None:
+            n = self.lib.mla_output_projection_workspace_bytes(ctypes.byref(dims), rows, d_model)
+            workspace = torch.empty(max(int(n), 16), dtype=torch.uint8, device=attn_out.device)
+        self._check(self.lib.mla_output_projection(ctypes.byref(dims), _ptr(attn_out), _ptr(W_O), rows, d_model,
+                                                   _ptr(y), _ptr(workspace), workspace.numel(), _stream(stream)))
+        return y
 
     def device_status(self, stream=None) -> int:
         """Synchronises the stream, returns and clears the device status bits."""

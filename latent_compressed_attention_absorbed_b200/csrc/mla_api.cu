@@ -182,7 +182,7 @@ using namespace mla;
 
 extern "C" {
 
-int mla_version(void) { return 100; }
+int mla_version(void) { return 101; }
 
 const char* mla_last_error(void) { return t_err; }
 
@@ -275,7 +275,8 @@ int mla_attend_latent(const mla_dims_t* dims, const void* q_hat, const mla_cache
                         workspace_bytes);
         workspace = align_ws(workspace, &workspace_bytes);
         e = sm100_attend(p, q_hat, cv, seqlens, o_lat, workspace, workspace_bytes, pairs,
-                         opts ? opts->overhead_tiles : -1, opts ? opts->min_tiles : 0, status, (cudaStream_t)stream);
+                         opts ? opts->overhead_tiles : -1, opts ? opts->min_tiles : 0, status, (cudaStream_t)stream,
+                         nullptr, false, true, nullptr, 0, opts);
     } else {
         e = generic_attend(p, q_hat, cv, seqlens, o_lat, status, (cudaStream_t)stream);
     }
@@ -363,7 +364,7 @@ int mla_decode_ex(const mla_dims_t* dims, const void* q_nope, const void* q_rope
             e = sm100_attend(p, q_hat, cv, seqlens, o_lat, ws + L.attend, L.total - L.attend, pairs,
                              opts ? opts->overhead_tiles : -1, opts ? opts->min_tiles : 0, status, st, &ev,
                              /*plan_ready=*/true, /*combine=*/!small, pf ? W_UV : nullptr,
-                             (size_t)p.H * p.d_v * p.d_c * 2);
+                             (size_t)p.H * p.d_v * p.d_c * 2, opts);
         ev.record(MLA_EV_COMBINE_DONE, st);
         if (e == cudaSuccess)
             e = small ? sm100_project_small(p, ws + L.attend, pairs, o_lat, W_UV, out, st)
@@ -387,6 +388,79 @@ int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_rope, c
                size_t workspace_bytes, mla_stream_t stream) {
     return mla_decode_ex(dims, q_nope, q_rope, W_UK, W_UV, cache, seqlens, B, q_len, out, workspace, workspace_bytes,
                          nullptr, stream);
+}
+
+size_t mla_append_from_hidden_workspace_bytes(const mla_dims_t* dims, int32_t B, int32_t n_tok, int32_t d_model) {
+    Problem p;
+    if (check_dims(dims, &p) || B < 0 || n_tok < 0 || d_model <= 0 || d_model % 64) return 0;
+    return append_hidden_workspace(B * n_tok, d_model) + kWsAlign;
+}
+
+int mla_append_from_hidden(const mla_dims_t* dims, const void* x, const void* W_A, const void* gamma,
+                           const int32_t* pos, int32_t B, int32_t n_tok, int32_t d_model, const mla_cache_t* cache,
+                           void* workspace, size_t workspace_bytes, mla_stream_t stream) {
+    t_err[0] = 0;
+    Problem p;
+    int rc = check_dims(dims, &p);
+    if (rc) return rc;
+    if (B < 0 || n_tok < 0 || d_model <= 0) return fail(MLA_ERR_ARG, "need B >= 0, n_tok >= 0, d_model > 0");
+    if (d_model % 64) return fail(MLA_ERR_SHAPE, "d_model must be a multiple of 64, got %d", d_model);
+    if (B == 0 || n_tok == 0) return MLA_OK;
+    if (!x || !W_A || !gamma || !pos) return fail(MLA_ERR_ARG, "NULL tensor pointer");
+    if (!aligned16(x) || !aligned16(W_A) || !aligned16(gamma) || !aligned4(pos))
+        return fail(MLA_ERR_ALIGN, "misaligned pointer");
+    p.B = B;
+    if (!sm100_linear_supported(p))
+        return fail(MLA_ERR_UNSUPPORTED,
+                    "mla_append_from_hidden needs a compute-capability 10.0 device, bf16 and the V3 head geometry");
+    CacheView cv;
+    rc = check_cache(p, cache, B, &cv);
+    if (rc) return rc;
+    const size_t need = append_hidden_workspace(B * n_tok, d_model) + kWsAlign;
+    if (!workspace || workspace_bytes < need || !aligned16(workspace))
+        return fail(MLA_ERR_WORKSPACE, "append workspace needs %zu bytes (16-byte aligned), got %zu", need,
+                    workspace_bytes);
+    workspace = align_ws(workspace, &workspace_bytes);
+    int* status = device_status_ptr();
+    if (!status) return fail(MLA_ERR_CUDA, "no CUDA device / status word");
+    t_path = "sm100";
+    cudaError_t e = sm100_append_hidden(p, x, W_A, gamma, pos, n_tok, d_model, cv, workspace, status,
+                                        (cudaStream_t)stream);
+    return e == cudaSuccess ? MLA_OK : cuda_fail(e, "append-from-hidden launch");
+}
+
+size_t mla_output_projection_workspace_bytes(const mla_dims_t* dims, int32_t rows, int32_t d_model) {
+    Problem p;
+    if (check_dims(dims, &p) || rows < 0 || d_model <= 0 || d_model % 64) return 0;
+    return output_projection_workspace(p, rows, d_model) + kWsAlign;
+}
+
+int mla_output_projection(const mla_dims_t* dims, const void* attn_out, const void* W_O, int32_t rows,
+                          int32_t d_model, void* y, void* workspace, size_t workspace_bytes, mla_stream_t stream) {
+    t_err[0] = 0;
+    Problem p;
+    int rc = check_dims(dims, &p);
+    if (rc) return rc;
+    if (rows < 0 || d_model <= 0) return fail(MLA_ERR_ARG, "need rows >= 0 and d_model > 0");
+    if (d_model % 64) return fail(MLA_ERR_SHAPE, "d_model must be a multiple of 64, got %d", d_model);
+    if (rows == 0) return MLA_OK;
+    if (!attn_out || !W_O || !y) return fail(MLA_ERR_ARG, "NULL tensor pointer");
+    if (!aligned16(attn_out) || !aligned16(W_O) || !aligned16(y)) return fail(MLA_ERR_ALIGN, "misaligned pointer");
+    p.B = rows;
+    if (!sm100_linear_supported(p))
+        return fail(MLA_ERR_UNSUPPORTED,
+                    "mla_output_projection needs a compute-capability 10.0 device, bf16 and the V3 head geometry");
+    const size_t need = output_projection_workspace(p, rows, d_model) + kWsAlign;
+    if (!workspace || workspace_bytes < need || !aligned16(workspace))
+        return fail(MLA_ERR_WORKSPACE, "output-projection workspace needs %zu bytes (16-byte aligned), got %zu", need,
+                    workspace_bytes);
+    workspace = align_ws(workspace, &workspace_bytes);
+    int* status = device_status_ptr();
+    if (!status) return fail(MLA_ERR_CUDA, "no CUDA device / status word");
+    t_path = "sm100";
+    cudaError_t e = sm100_output_projection(p, attn_out, W_O, rows, d_model, y, workspace, status,
+                                            (cudaStream_t)stream);
+    return e == cudaSuccess ? MLA_OK : cuda_fail(e, "output-projection launch");
 }
 
 int mla_device_status(mla_stream_t stream, int32_t* status) {

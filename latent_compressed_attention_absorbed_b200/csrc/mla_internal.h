@@ -86,7 +86,7 @@ cudaError_t sm100_attend(const Problem& p, const void* q_hat, const CacheView& c
                          void* o_lat, void* workspace, size_t ws_bytes, int num_pairs, int overhead_tiles,
                          int min_tiles, int* status, cudaStream_t st, const Events* events = nullptr,
                          bool plan_ready = false, bool combine = true, const void* prefetch = nullptr,
-                         size_t prefetch_bytes = 0);
+                         size_t prefetch_bytes = 0, const mla_decode_opts_t* opts = nullptr);
 cudaError_t sm100_project(const Problem& p, const void* o_lat, const void* W_UV, int rows, void* out,
                           cudaStream_t st);
 // Small batches: matrix-vector kernels.  The project step (B * q_len <= 8)
@@ -100,6 +100,16 @@ cudaError_t sm100_absorb_small(const Problem& p, const void* q_nope, const void*
 cudaError_t sm100_project_small(const Problem& p, void* attend_workspace, int num_pairs, const void* o_lat,
                                 const void* W_UV, void* out, cudaStream_t st);
 size_t sm100_attend_workspace_bytes(const Problem& p, int num_pairs);
+// Projections around the attention step (bf16, V3 geometry): the cache append
+// from the block input and the output projection.
+bool sm100_linear_supported(const Problem& p);
+size_t append_hidden_workspace(int rows, int d_model);
+size_t output_projection_workspace(const Problem& p, int rows, int d_model);
+cudaError_t sm100_append_hidden(const Problem& p, const void* x, const void* W_A, const void* gamma,
+                                const int32_t* pos, int n_tok, int d_model, const CacheView& cache, void* ws,
+                                int* status, cudaStream_t st);
+cudaError_t sm100_output_projection(const Problem& p, const void* attn_out, const void* W_O, int rows, int d_model,
+                                    void* y, void* ws, int* status, cudaStream_t st);
 int sm100_default_pairs();
 
 }  // namespace mla

@@ -10,6 +10,7 @@
 
 #include "mla_internal.h"
 #include "mla_rope.cuh"
+#include "sm100_host.h"
 #include "sm100_attend.cuh"
 #include "sm100_gemm.cuh"
 #include "sm100_gemv.cuh"
@@ -49,38 +50,6 @@ using namespace sm100;
 
 namespace {
 
-// ------------------------------------------------------------------ tensor maps
-
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
-    return fn;
-}
-
-// 3-D bf16 map: dims (d0 innermost, d1, d2), byte strides of d1 and d2, box (b0, b1, b2).
-bool make_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1, uint64_t s2,
-              uint32_t b0, uint32_t b1, uint32_t b2, CUtensorMapSwizzle sw) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    const cuuint64_t dims[3] = {d0, d1, d2};
-    const cuuint64_t strides[2] = {s1, s2};
-    const cuuint32_t box[3] = {b0, b1, b2};
-    const cuuint32_t estr[3] = {1, 1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 // ------------------------------------------------------------------ append
 
 // One warp per new token: 16-byte copies of the 512 latent values and the
@@ -111,51 +80,8 @@ __global__ void append_v3_kernel(const __nv_bfloat16* __restrict__ c_kv, const _
     MLA_KT(kKtAppend, 2);
 }
 
-// Opt a kernel into more than 48 KB of dynamic shared memory, once per device
-// and call site (`done` is that site's own flag array), so that later calls,
-// including ones under stream capture, make no attribute calls.
-constexpr int kMaxDev = 64;
-template <typename K>
-cudaError_t set_smem(K kernel, int bytes, bool (&done)[kMaxDev]) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < kMaxDev && done[dev]) return cudaSuccess;
-    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (e == cudaSuccess && dev >= 0 && dev < kMaxDev) done[dev] = true;
-    return e;
-}
 bool g_smem_absorb[kMaxDev], g_smem_project[kMaxDev], g_smem_attend[kMaxDev];
 bool g_smem_absorb_gemv[4][kMaxDev], g_smem_project_gemv[4][kMaxDev];
-
-// Launch with programmatic dependent launch allowed: the kernel may start
-// while the previous kernel on the stream is finishing; it calls
-// griddepcontrol.wait before touching anything that kernel may write.
-template <typename... KArgs, typename... Args>
-cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, int cluster_x,
-                       Args&&... args) {
-    cudaLaunchConfig_t cfg;
-    memset(&cfg, 0, sizeof(cfg));
-    cfg.gridDim = grid;
-    cfg.blockDim = block;
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[2];
-    int n = 0;
-    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[n].val.programmaticStreamSerializationAllowed = 1;
-    ++n;
-    if (cluster_x > 1) {
-        attr[n].id = cudaLaunchAttributeClusterDimension;
-        attr[n].val.clusterDim.x = cluster_x;
-        attr[n].val.clusterDim.y = 1;
-        attr[n].val.clusterDim.z = 1;
-        ++n;
-    }
-    cfg.attrs = attr;
-    cfg.numAttrs = n;
-    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
-}
 
 constexpr int kAbsorbStages = 2;
 // Rows of the A tile a GEMM CTA loads: all 128 when the batch fills them,
@@ -344,7 +270,7 @@ size_t sm100_attend_workspace_bytes(const Problem& p, int num_pairs) {
 cudaError_t sm100_attend(const Problem& p, const void* q_hat, const CacheView& cache, const int32_t* seqlens,
                          void* o_lat, void* workspace, size_t ws_bytes, int num_pairs, int overhead_tiles,
                          int min_tiles, int* status, cudaStream_t st, const Events* events, bool plan_ready,
-                         bool combine, const void* prefetch, size_t prefetch_bytes) {
+                         bool combine, const void* prefetch, size_t prefetch_bytes, const mla_decode_opts_t* opts) {
     const int clusters = attend_clusters(num_pairs, p.q_len);
     if (clusters / p.q_len > kPlanMaxGroups) return cudaErrorInvalidValue;
     size_t off_part, off_lse;
@@ -352,16 +278,12 @@ cudaError_t sm100_attend(const Problem& p, const void* q_hat, const CacheView& c
     if (ws_bytes < need) return cudaErrorInvalidValue;
     char* ws = static_cast<char*>(workspace);
     Plan* plan = reinterpret_cast<Plan*>(ws);
-    // Cache as [B][T_max][576]: latent boxes of 64 columns (SW128), RoPE half
-    // boxes of 32 columns (SW64), 64 keys each, and 256-column boxes for the
-    // L2 prefetch.
-    CUtensorMap mLat, mRope, mPf, mQR;
+    // The cache as [B][T_max][576]: boxes of 64 columns x 64 keys (SW128); the
+    // scoring CTA loads all nine of a row tile, the accumulating CTA the eight
+    // latent ones.
+    CUtensorMap mRow;
     const uint64_t sb = (uint64_t)cache.stride_b * 2, stt = (uint64_t)cache.stride_t * 2;
-    if (!make_map(&mLat, cache.data, kRow, cache.T_max, p.B, stt, sb, 64, kNk, 1, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&mRope, cache.data, kRow, cache.T_max, p.B, stt, sb, kHalfRope, kNk, 1, CU_TENSOR_MAP_SWIZZLE_64B) ||
-        !make_map(&mPf, cache.data, kRow, cache.T_max, p.B, stt, sb, kHalfLat, kNk, 1, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !make_map(&mQR, q_hat, kRow, kHeads, (uint64_t)p.B * p.q_len, kRow * 2, (uint64_t)kHeads * kRow * 2, kHalfRope,
-                  kHeads, 1, CU_TENSOR_MAP_SWIZZLE_64B))
+    if (!make_map(&mRow, cache.data, kRow, cache.T_max, p.B, stt, sb, 64, kNk, 1, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
 
     cudaError_t e;
@@ -387,9 +309,15 @@ cudaError_t sm100_attend(const Problem& p, const void* q_hat, const CacheView& c
     a.part_o = reinterpret_cast<float*>(ws + off_part);
     a.part_lse = reinterpret_cast<float*>(ws + off_lse);
     a.status = status;
+    a.wait_limit_ns = (opts && opts->wait_limit_ns > 0) ? (uint64_t)opts->wait_limit_ns : MLA_WAIT_LIMIT_NS;
+    a.withhold_tile = (opts && opts->withhold_tile > 0) ? opts->withhold_tile : -1;
+    a.cache = static_cast<const uint8_t*>(cache.data);
+    a.stride_b = cache.stride_b * 2;
+    a.stride_t = cache.stride_t * 2;
+    a.T_max = cache.T_max;
 
     if (events) events->record(MLA_EV_ATTEND_BEGIN, st);
-    e = launch_pdl(mla_attend_kernel, dim3(clusters * 2), dim3(kAttThreads), kAttSmem, st, 2, mLat, mRope, mPf, mQR, a);
+    e = launch_pdl(mla_attend_kernel, dim3(clusters * 2), dim3(kAttThreads), kAttSmem, st, 2, mRow, a);
     if (e != cudaSuccess) return e;
     if (events) events->record(MLA_EV_ATTEND_END, st);
 

@@ -10,17 +10,24 @@
 // aggregate sum_j p_j c_KV,j before W_UV; m.lsln.cn section 2.1: softmax over
 // the whole history.)
 //
-// Work split.  The fp32 accumulator of 128 heads x 512 latent columns would
-// fill all 512 TMEM columns of an SM, and an M = 64 MMA runs at half the
-// tensor rate, so a CTA keeps all 128 heads (M = 128) and a cluster of two
-// CTAs splits the 576-wide cache row: CTA r loads and multiplies latent
-// columns 256r..256r+255 and RoPE columns 32r..32r+31 of every tile (the
-// cache crosses HBM and L2 once).  Each CTA computes a partial S over its
-// 288 columns, scales it to log2 units and rounds it to fp16; the pair swaps
-// the rounded partials through distributed shared memory (one bulk copy per
-// warp), both add the two halves (fp32 addition is commutative, so both CTAs
-// see the same S), run the same online softmax, and each accumulates its
-// 256 latent columns of O in TMEM.
+// Work split.  One query token's 128 heads are the M dimension of every
+// MMA.  Its fp32 output accumulator, 128 heads x 512 latent columns, fills
+// the 512 TMEM columns of an SM, so a cluster of two CTAs shares the work:
+//   * the scoring CTA (rank 0) holds Q-hat (576 bf16 per head) in TMEM,
+//     loads whole cache rows (576 columns) for 64 keys at a time and computes
+//     the exact fp32 scores S (36 MMAs of K = 16 into one of two TMEM
+//     buffers), runs the online softmax, and streams P (bf16) and each row's
+//     rescale factor and running sum to the accumulating CTA: the softmax
+//     warps write them into a local staging slot and one lane per TMEM
+//     quarter bulk-copies the quarter's rows into the peer's slot;
+//   * the accumulating CTA (rank 1) loads the latent part of the same rows
+//     (an L2 hit) and accumulates O += P . C_KV with P as the shared-memory
+//     A operand (two MMAs of N = 256 per K step), rescales O's rows when the
+//     scorer's running maximum grew, and writes the normalised o_lat or the
+//     split partial at the end of a piece.
+// The traffic between the pair is one way (18 KB per 64 keys) through a
+// ring of three slots, so its latency is hidden; the scorer's stage is
+// released as soon as its score MMAs complete.
 //
 // Scheduling (split-KV).  Sequences are cut into 64-key tiles.  The clusters
 // form groups of q_len (cluster c: group c / q_len, query token c % q_len);
@@ -32,21 +39,19 @@
 // groups writes fp32 partials plus a base-2 LSE per head and token, merged by
 // the combine kernel.
 //
-// Roles per CTA (512 threads; warps 12-15 are the second softmax warp of each
-// quarter, warp 11 is idle):
-//   warp 0     TMA producer (stage ring, L2 prefetch of the tiles ahead);
-//   warp 1     TMEM owner and issuer of the score MMAs (S);
-//   warp 10    issuer of the P.V MMAs (O), as soon as P is published;
-//   warps 2-5, softmax, two warps per TMEM lane quarter (32 keys each): add
-//   12-15      the two partial scores, online softmax, P into TMEM, rescale /
-//              normalise O, write o_lat or split partials;
-//   warps 6-9  exchange: read partial S out of TMEM, publish it (local copy
-//              for the softmax warps, bulk copy to the peer), load Q-hat.
-// Warp w reaches TMEM lanes 32*(w%4)..+31; lane l of warp w owns head
-// 32*(w%4)+l, a whole score row.  Every wait is bounded; on expiry the
-// kernel flags MLA_STATUS_TIMEOUT, stops issuing work and tears down
-// normally (the two softmax warps of a quarter, which meet on a named
-// barrier, decide together whether to stop, so neither is left waiting).
+// Roles (512 threads; warp w reaches TMEM lanes 32*(w%4)..+31, and lane l
+// of a warp owns head 32*(w%4)+l, a whole row):
+//   scorer:      warp 0 TMA producer; warp 1 TMEM owner and S issuer;
+//                warps 2-5 and 12-15 softmax, two per TMEM quarter (32 keys
+//                each); warps 6-9 load Q-hat into TMEM once per piece;
+//   accumulator: warp 0 TMA producer; warp 1 TMEM owner and O issuer;
+//                warps 2-5 and 12-15 rescale / epilogue, two per quarter
+//                (256 columns each); warp 10 returns consumed P slots.
+// Every wait is bounded; on expiry the kernel flags MLA_STATUS_TIMEOUT,
+// stops issuing work, drains what it has in flight (stage loads, MMAs, the
+// peer's copies into its shared memory) and tears down normally (the two
+// softmax warps of a quarter, which meet on a named barrier, decide together
+// whether to stop, so neither is left waiting).
 #pragma once
 
 #include <cuda_bf16.h>
@@ -65,71 +70,85 @@ constexpr int kHeads = 128;  // heads of a token (M of every MMA)
 constexpr int kLat = 512;    // d_c
 constexpr int kRope = 64;    // d_r
 constexpr int kRow = kLat + kRope;
-constexpr int kHalfLat = 256;
-constexpr int kHalfRope = 32;
 
 // Shared-memory map (offsets from a 1024-aligned base).
-//   stages: ring of this CTA's half tiles: 4 SW128 chunks of 64 keys x 64
-//           latent columns, then 64 keys x 32 RoPE columns (SW64);
-//   Own:    two buffers of this CTA's partial scores, 128 x 64 fp16 (rows of
-//           128 bytes, 16-byte chunks swizzled by row), read by the local
-//           softmax warps and bulk-copied to the peer's X buffer;
-//   X:      two buffers receiving the peer's partial scores (same layout);
-//   QR:     this CTA's RoPE half of Q-hat, 128 heads x 32 bf16 (SW64).
-constexpr int kChunk = kNk * 128;                     // 8192
-constexpr int kRopeChunk = kNk * 64;                  // 4096
-constexpr int kStageBytes = 4 * kChunk + kRopeChunk;  // 36864
-constexpr int kStages = 4;
-#ifndef MLA_PREFETCH_TILES
-#define MLA_PREFETCH_TILES 6
+// Scoring CTA (cluster rank 0):
+//   stages:  kSStages whole cache rows of 64 keys: 9 SW128 chunks of 64 keys
+//            x 64 columns (latent 0..511, then RoPE 512..575), 72 KB each;
+//   staging: kPSlots local copies of the accumulator's P slots (same layout),
+//            written by the softmax warps and bulk-copied to the peer;
+//   red, flags: the softmax pairs' row maxima / sums and their status.
+// Accumulating CTA (cluster rank 1):
+//   vstages: kVStages latent parts of 64 keys (8 SW128 chunks), 64 KB each;
+//   pslots:  kPSlots slots, each P of 128 heads x 64 keys (bf16, SW128,
+//            K-major: the A operand of the O MMA) followed by 16 bytes per
+//            head: the rescale factor of O and the two halves' sums of p.
+constexpr int kChunk = kNk * 128;            // 8192: 64 keys x 64 columns
+constexpr int kSStages = 2;
+constexpr int kSStageBytes = 9 * kChunk;     // 73728
+constexpr int kVStages = 2;
+constexpr int kVStageBytes = 8 * kChunk;     // 65536
+constexpr int kPSlots = 3;
+constexpr int kPData = kHeads * 128;         // 16384
+constexpr int kPSlotBytes = kPData + kHeads * 16;  // 18432
+constexpr int kOffSStages = 0;
+constexpr int kOffStaging = kSStages * kSStageBytes;
+constexpr int kOffRed = kOffStaging + kPSlots * kPSlotBytes;  // [2 tiles][2 halves][128 rows] fp32
+constexpr int kOffFlags = kOffRed + 2 * 2 * kHeads * 4;       // [2 tiles][4 quarters][2] int, twice
+constexpr int kScorerEnd = kOffFlags + 2 * 2 * 4 * 2 * 4;
+#ifndef MLA_SCORE_PREFETCH
+#define MLA_SCORE_PREFETCH 0
 #endif
-constexpr int kPrefetch = MLA_PREFETCH_TILES;  // tiles prefetched into L2 ahead of the stage loads
-constexpr int kXBytes = kHeads * 128;                 // 16384
-constexpr int kOffStages = 0;
-constexpr int kOffOwn = kOffStages + kStages * kStageBytes;
-constexpr int kOffX = kOffOwn + 2 * kXBytes;
-constexpr int kQRBytes = kHeads * 64;                  // 8192
-constexpr int kOffQR = kOffX + 2 * kXBytes;
-constexpr int kOffRed = kOffQR + kQRBytes;            // softmax pair exchange: [2][2][128] fp32
-constexpr int kOffFlags = kOffRed + 2 * 2 * kHeads * 4;  // softmax pair status: [2][4 quarters][2] int
-constexpr int kOffBars = kOffFlags + 2 * 4 * 2 * 4;
-constexpr int kAttSmem = kOffBars + 256 + 1024;
+// Row tiles the scorer prefetches into L2 ahead of its stage loads (0: off;
+// 4 and 8 tiles measured slower than none on B200, where the two-stage ring
+// of each scorer already keeps HBM busy).
+constexpr int kScorePrefetch = MLA_SCORE_PREFETCH;
+constexpr int kOffVStages = 0;
+constexpr int kOffPSlots = kVStages * kVStageBytes;
+constexpr int kAccumEnd = kOffPSlots + kPSlots * kPSlotBytes;
+constexpr int kOffBars = (kScorerEnd > kAccumEnd ? kScorerEnd : kAccumEnd);
+constexpr int kBarBytes = 512;  // barrier block: the mbarriers, then the TMEM base and the abort flag
+constexpr int kAttSmem = kOffBars + kBarBytes + 1024;
+static_assert(kOffPSlots % 1024 == 0 && kPSlotBytes % 1024 == 0, "P slots must start on 1024-byte boundaries");
 static_assert(kAttSmem <= 232448, "attention kernel shared memory exceeds 227 KB");
 
-// Tensor-memory map: 512 columns of 32 bits, lane = head.
+// Tensor-memory maps: 512 columns of 32 bits, lane = head.
 constexpr int kTmemCols = 512;
-constexpr int kTmemO = 0;     // O: 256 fp32 latent columns of this CTA's half
-constexpr int kTmemS = 256;   // S: 64 fp32 partial scores
-constexpr int kTmemP = 320;   // P: two buffers of 64 bf16 probabilities, two per column
-constexpr int kTmemQ = 384;   // Q-hat latent half: 256 bf16, two per column (128 columns)
+constexpr int kTmemQ = 0;    // scorer: Q-hat, 576 bf16, two per column (288 columns)
+constexpr int kTmemS = 384;  // scorer: two S buffers of 64 fp32 columns (384, 448)
+constexpr int kTmemO = 0;    // accumulator: O, 512 fp32 latent columns
 constexpr int kAttThreads = 512;
 
 // Barrier indices (8 bytes each) inside the barrier block.
 enum {
-    kBarFull0 = 0,
-    kBarEmpty0 = kBarFull0 + kStages,
-    kBarQFull = kBarEmpty0 + kStages,  // Q-hat of the next piece loaded (4 exchange warps + RoPE-half TMA)
-    kBarSFull,                         // S(g) complete (MMA commit)
-    kBarSFree,                         // S(g) read out of TMEM (4 exchange warps)
-    kBarPFull0,                        // P(g) in TMEM buffer g%2 (4 softmax warps)
-    kBarPFree0 = kBarPFull0 + 2,       // O(g) complete: P buffer g%2 (and O) may be touched (MMA commit)
-    kBarOwnFull0 = kBarPFree0 + 2,     // own partial g in Own[g%2] (4 exchange warps)
-    kBarOwnFree0 = kBarOwnFull0 + 2,   // Own[g%2] read by the softmax warps (4)
-    kBarXFull0 = kBarOwnFree0 + 2,     // peer's partial g landed in X[g%2] (tx)
-    kBarXFree0 = kBarXFull0 + 2,       // the peer has read what we sent into its X[g%2] (4, remote)
-    kBarOFull = kBarXFree0 + 2,        // last O of a piece complete (MMA commit)
-    kBarOFree,                         // O read by the epilogue (8 softmax warps)
+    // scorer
+    kBarFull0 = 0,                      // stage loaded (tx)
+    kBarEmpty0 = kBarFull0 + kSStages,  // stage read by S (MMA commit)
+    kBarSFull0 = kBarEmpty0 + kSStages, // S(g) in buffer g%2 (MMA commit)
+    kBarSFree0 = kBarSFull0 + 2,        // S buffer read by the 8 softmax warps
+    kBarQFull = kBarSFree0 + 2,         // Q-hat of a piece in TMEM (4 loader warps)
+    kBarQRead,                          // the last S of a piece complete: Q-hat may be replaced (MMA commit)
+    kBarSlotFree0 = kBarQRead + 1,      // accumulator's P slot consumed (remote arrive)
+    // accumulator
+    kBarVFull0 = kBarSlotFree0 + kPSlots,  // latent part loaded (tx)
+    kBarVEmpty0 = kBarVFull0 + kVStages,   // latent part read by O (MMA commit)
+    kBarPFull0 = kBarVEmpty0 + kVStages,   // P(g) and its row data landed (tx, from the scorer)
+    kBarPDone0 = kBarPFull0 + kPSlots,     // O(g) complete: the slot was read (MMA commit)
+    kBarRescaled0 = kBarPDone0 + kPSlots,  // O rows rescaled for tile g if needed (8 epilogue warps)
+    kBarOFull = kBarRescaled0 + kPSlots,   // last O of a piece complete (MMA commit)
+    kBarOFree,                             // O read by the epilogue (8 warps)
+    // both
+    kBarDrain,                             // every MMA of the issuer complete (teardown)
     kNumBars
 };
-static_assert(8 * (kNumBars + 2) <= 256, "barrier block too small");
+static_assert(8 * (kNumBars + 2) <= kBarBytes, "barrier block too small");
 
 // Optional timing trace (compile with -DMLA_TRACE): global-timer stamps (ns)
 // of both CTAs of one cluster at fixed points of every tile, read back by
-// mla_trace_read.  Events: 0 tile loads issued, 1 S issued, 2 O issued,
-// 3 S read by the exchange warps, 4 own partial published, 5 both partials
-// available to the softmax warps, 6 P published, 7 piece epilogue done,
-// 8 row max, 9 P computed, 10 tile data seen by the MMA warp, 11..13 P
-// published by warps 3, 4, 5.
+// mla_trace_read.  Scorer: 0 stage loads issued, 14 S issue start, 1 S
+// issued, 3 S read by the softmax warps, 4 P handed to the bulk copies.
+// Accumulator: 0 stage loads issued, 5 O rows rescaled (or checked), 15 O
+// issue start, 2 O issued, 7 piece epilogue done.
 #ifdef MLA_TRACE
 #ifndef MLA_TRACE_CLUSTER
 #define MLA_TRACE_CLUSTER 0
@@ -148,14 +167,14 @@ __device__ unsigned long long g_mla_trace[2][kTraceTiles][16];
 constexpr int kTraceAllClusters = 256;
 __device__ unsigned long long g_mla_trace_all[kTraceAllClusters][2][24];
 enum {
-    kTwFull,      // S issuer: tile data
-    kTwSFree,     // S issuer: previous S read out of TMEM
+    kTwFull,      // S issuer: stage loaded / O issuer: latent part loaded
+    kTwSFree,     // S issuer: S buffer read out of TMEM
     kTwQFull,     // S issuer: Q-hat of a piece
-    kTwSFull,     // exchange: S complete
-    kTwOwnFree,   // exchange: buffers of tile h-2 released (own and peer)
-    kTwXFull,     // softmax: own and peer partials
-    kTwPFree,     // softmax: P buffer released by O(g-2) (and O ready for a rescale)
-    kTwPFull,     // O issuer: P published
+    kTwSFull,     // (unused)
+    kTwOwnFree,   // (unused)
+    kTwXFull,     // softmax: S complete / epilogue: P slot landed
+    kTwPFree,     // softmax: the peer's P slot consumed
+    kTwPFull,     // O issuer: P slot landed, rows rescaled
     kTwOFree,     // O issuer: previous piece's O read
     kTwEmpty,     // producer: stage released
     kTwN
@@ -300,35 +319,48 @@ struct AttendArgs {
     float* part_o;                // [slots][64 column octets][128 heads][8]
     float* part_lse;              // [slots][128]
     int* status;
+    uint64_t wait_limit_ns;       // time limit of every barrier wait
+    int withhold_tile;            // test hook (>= 0): the loaders stop before this tile (see mla.h)
+    const uint8_t* cache;         // the cache rows, for the L2 prefetch of whole row tiles
+    int64_t stride_b, stride_t;   // (bytes; the prefetch runs only when a tile's rows are contiguous)
+    int T_max;
 };
 
 // Byte offset of 16-byte chunk c of row r in a buffer of 128-byte rows whose
-// chunks are permuted by row (c ^ (r % 8)), the SW128 pattern: the 8 rows a
-// quarter-warp touches at once land in 8 different bank groups.
+// chunks are permuted by row (c ^ (r % 8)): the SW128 layout the tensor core
+// reads (K-major, 1024-byte groups of 8 rows), and the 8 rows a quarter-warp
+// touches at once land in 8 different bank groups.
 __device__ __forceinline__ uint32_t sw128(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
 
-// mapLat: cache [B][T_max][576] bf16, box 64 columns x 64 keys, SW128.
-// mapRope: same tensor, box 32 columns x 64 keys, SW64.
-// mapPf: the cache again, box 256 columns x 64 keys, no swizzle (L2 prefetch only).
-// mapQR: q_hat [U][128][576] bf16, box 32 columns x 128 heads, SW64.
+// Rows at or beyond the sequence length hold no cached token: zero `nchunks`
+// SW128 chunks of 64 keys from row r0 on (one warp), so that masked rows can
+// inject no NaN / Inf through p = 0.
+__device__ __forceinline__ void zero_rows(uint32_t tile, int nchunks, int r0, int lane) {
+    for (int row = r0 + (lane >> 3); row < kNk; row += 4)
+        for (int c = 0; c < nchunks; ++c) st_shared_v4(tile + c * kChunk + row * 128 + (lane & 7) * 16, 0, 0, 0, 0);
+    fence_proxy_async_smem();
+}
+
+// mapRow: the cache [B][T_max][576] bf16, box 64 columns x 64 keys, SW128.
 __global__ void __launch_bounds__(kAttThreads, 1)
-    mla_attend_kernel(const __grid_constant__ CUtensorMap mapLat, const __grid_constant__ CUtensorMap mapRope,
-                      const __grid_constant__ CUtensorMap mapPf, const __grid_constant__ CUtensorMap mapQR,
-                      AttendArgs args) {
+    mla_attend_kernel(const __grid_constant__ CUtensorMap mapRow, AttendArgs args) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t* base_ptr = smem_raw + (base - raw);
     auto bar = [&](int i) { return base + kOffBars + 8u * i; };
     const uint32_t tmem_slot = bar(kNumBars);
+    const uint32_t abort_addr = bar(kNumBars + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(base_ptr + kOffBars + 8 * (kNumBars + 1));
+    const uint64_t lim = args.wait_limit_ns;
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const uint32_t r = cluster_ctarank() & 1;  // latent half of this CTA
-    const uint32_t peer = r ^ 1;
+    const uint32_t rank = cluster_ctarank() & 1;  // 0: scorer, 1: accumulator
+    const uint32_t peer = rank ^ 1;
     const int cl = (int)cluster_id_x();
     const int q_len = args.q_len;
     const int grp = cl / q_len, qi = cl % q_len;
+    [[maybe_unused]] const uint32_t r = rank;  // for the trace macros
 
     if (threadIdx.x == 0) MLA_TRACE_POINT(0, kTraceProlog);
     if (threadIdx.x == 0) MLA_TRACE_ALL(0, global_timer_ns());
@@ -338,37 +370,36 @@ __global__ void __launch_bounds__(kAttThreads, 1)
 #pragma unroll
     for (int i = 0; i < kTwN; ++i) tw_acc[i] = 0;
 #endif
-#ifdef MLA_TRACE
     if (threadIdx.x == 0) {
-        unsigned smid;
-        asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
-        MLA_TRACE_ALL(8, smid);
-    }
-#endif
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
-            mbar_init(bar(kBarFull0 + s), 1);
-            mbar_init(bar(kBarEmpty0 + s), 1);
+        if (rank == 0) {
+            for (int s = 0; s < kSStages; ++s) {
+                mbar_init(bar(kBarFull0 + s), 1);
+                mbar_init(bar(kBarEmpty0 + s), 1);
+            }
+            for (int s = 0; s < 2; ++s) {
+                mbar_init(bar(kBarSFull0 + s), 1);
+                mbar_init(bar(kBarSFree0 + s), 8);
+            }
+            mbar_init(bar(kBarQFull), 4);
+            mbar_init(bar(kBarQRead), 1);
+            for (int s = 0; s < kPSlots; ++s) mbar_init(bar(kBarSlotFree0 + s), 1);
+        } else {
+            for (int s = 0; s < kVStages; ++s) {
+                mbar_init(bar(kBarVFull0 + s), 1);
+                mbar_init(bar(kBarVEmpty0 + s), 1);
+            }
+            for (int s = 0; s < kPSlots; ++s) {
+                mbar_init(bar(kBarPFull0 + s), 1);
+                mbar_init(bar(kBarPDone0 + s), 1);
+                mbar_init(bar(kBarRescaled0 + s), 8);
+            }
+            mbar_init(bar(kBarOFull), 1);
+            mbar_init(bar(kBarOFree), 8);
         }
-        mbar_init(bar(kBarQFull), 5);
-        mbar_init(bar(kBarSFull), 1);
-        mbar_init(bar(kBarSFree), 4);
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(bar(kBarPFull0 + s), 8);
-            mbar_init(bar(kBarPFree0 + s), 1);
-            mbar_init(bar(kBarOwnFull0 + s), 4);
-            mbar_init(bar(kBarOwnFree0 + s), 8);
-            mbar_init(bar(kBarXFull0 + s), 1);
-            mbar_init(bar(kBarXFree0 + s), 8);
-        }
-        mbar_init(bar(kBarOFull), 1);
-        mbar_init(bar(kBarOFree), 8);
+        mbar_init(bar(kBarDrain), 1);
         *abort_flag = 0;
         fence_mbar_init();
-        prefetch_tensormap(&mapLat);
-        prefetch_tensormap(&mapRope);
-        prefetch_tensormap(&mapPf);
-        prefetch_tensormap(&mapQR);
+        prefetch_tensormap(&mapRow);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, kTmemCols);
@@ -378,13 +409,11 @@ __global__ void __launch_bounds__(kAttThreads, 1)
     // The peer's barriers must be initialised before any remote access.
     cluster_sync();
     tc_fence_after();
-    if (threadIdx.x == 0) MLA_TRACE_POINT(1, kTraceProlog);
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(base_ptr + kOffBars + 8 * kNumBars);
     // The set-up above overlaps the previous kernel; the plan, Q-hat and the
     // cache are read only once it has completed.
     pdl_wait();
     if (threadIdx.x == 0) pdl_trigger();
-    if (threadIdx.x == 0) MLA_TRACE_POINT(2, kTraceProlog);
     if (threadIdx.x == 0) MLA_TRACE_ALL(1, global_timer_ns());
     MLA_KT(kKtAttend, 1);
     const bool active = grp < args.plan->groups;
@@ -400,113 +429,91 @@ __global__ void __launch_bounds__(kAttThreads, 1)
     }
 
     const int quarter = warp & 3;
-    const int m = quarter * 32 + lane;                          // head / TMEM lane (warps 2..9)
+    const int m = quarter * 32 + lane;                          // head / TMEM lane
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;  // the warp's TMEM subpartition
+    const bool softmax_warp = (warp >= 2 && warp <= 5) || warp >= 12;
+    const int kh = warp >= 12 ? 1 : 0;  // key half (scorer) / column half (accumulator)
+    int n_loads = 0;                    // stage loads issued (producer lane), for the teardown
 
     if (!active) {
         // idle cluster (the cluster count is not a multiple of q_len)
     } else if (warp == 0) {
-        // ======================================================== TMA producer (runs up to kStages tiles ahead)
-        // Tiles kPrefetch ahead of the loads are prefetched into L2, so that a
-        // stage, once freed, refills at L2 rather than HBM latency.  (Issuing the
-        // first loads ahead of the first prefetches measured slower: the early
-        // burst of prefetches keeps HBM busy while the pipeline fills.)
+        // ======================================================== TMA producer (both CTAs)
+        // scorer: whole rows (9 chunks) into kSStages stages, released by S;
+        // accumulator: latent parts (8 chunks) into kVStages stages, released by O.
         if (lane == 0) {
+            const int nst = rank == 0 ? kSStages : kVStages;
+            const int nch = rank == 0 ? 9 : 8;
+            const int sbytes = rank == 0 ? kSStageBytes : kVStageBytes;
+            const int full0 = rank == 0 ? kBarFull0 : kBarVFull0;
+            const int empty0 = rank == 0 ? kBarEmpty0 : kBarVEmpty0;
             TileWalk w, wp;
             w.init(args.plan, grp);
             wp = w;
-            for (int i = 0; i < kPrefetch && wp.valid; ++i) {
-                tma_prefetch_3d(&mapPf, kHalfLat * r, wp.t * kNk, wp.seq);
-                tma_prefetch_3d(&mapRope, kLat + kHalfRope * r, wp.t * kNk, wp.seq);
-                wp.advance();
-            }
+            // The scorer prefetches whole row tiles into L2 a few tiles ahead
+            // of its stage loads (a tile is contiguous when rows are packed);
+            // the accumulator's loads of the same tiles then hit L2.
+            const bool pf = rank == 0 && kScorePrefetch > 0 && args.stride_t == (int64_t)kRow * 2;
+            auto prefetch_tile = [&](const TileWalk& t) {
+                const int rows = args.T_max - t.t * kNk < kNk ? args.T_max - t.t * kNk : kNk;
+                if (rows > 0)
+                    prefetch_l2_bulk(args.cache + (size_t)t.seq * args.stride_b + (size_t)t.t * kNk * args.stride_t,
+                                     (uint32_t)rows * kRow * 2);
+            };
+            if (pf)
+                for (int i = 0; i < kScorePrefetch && wp.valid; ++i, wp.advance()) prefetch_tile(wp);
             for (int n = 0; w.valid && !*abort_flag; ++n, w.advance()) {
-                if (kPrefetch > 0 && wp.valid) {
-                    // A later piece's Q-hat (147 KB, contiguous) goes into L2 as the
-                    // look-ahead enters it, ahead of its reload: each CTA of the
-                    // pair prefetches one half, 8 KB a request.
-                    if (wp.first() && wp.seg > 0) {
-                        constexpr uint32_t kQBytes = kHeads * kRow * 2, kPiece = 8192;
-                        const uint8_t* q = reinterpret_cast<const uint8_t*>(args.q_hat) +
-                                           (size_t)(wp.seq * q_len + qi) * kQBytes;
-                        for (uint32_t off = r * (kQBytes / 2); off < (r + 1) * (kQBytes / 2); off += kPiece)
-                            prefetch_l2_bulk(q + off, kPiece);
-                    }
-                    tma_prefetch_3d(&mapPf, kHalfLat * r, wp.t * kNk, wp.seq);
-                    tma_prefetch_3d(&mapRope, kLat + kHalfRope * r, wp.t * kNk, wp.seq);
+                // Test hook: stop before tile `withhold_tile`, which is then never
+                // loaded, so that a bounded wait for it runs out.
+                if (n == args.withhold_tile) break;
+                if (pf && wp.valid) {
+                    prefetch_tile(wp);
                     wp.advance();
                 }
-                const int st = n % kStages;
-                if (n >= kStages && !MLA_TW(kTwEmpty, mbar_wait(bar(kBarEmpty0 + st), ((n / kStages) - 1) & 1))) {
+                const int st = n % nst;
+                if (n >= nst && !MLA_TW(kTwEmpty, mbar_wait(bar(empty0 + st), ((n / nst) - 1) & 1, lim))) {
                     *abort_flag = 1;
                     break;
                 }
-                const uint32_t dst = base + kOffStages + st * kStageBytes;
-                mbar_arrive_expect_tx(bar(kBarFull0 + st), kStageBytes);
-#pragma unroll
-                for (int c = 0; c < 4; ++c)
-                    tma_load_3d(dst + c * kChunk, &mapLat, bar(kBarFull0 + st), kHalfLat * r + 64 * c, w.t * kNk, w.seq);
-                tma_load_3d(dst + 4 * kChunk, &mapRope, bar(kBarFull0 + st), kLat + kHalfRope * r, w.t * kNk, w.seq);
+                const uint32_t dst = base + st * sbytes;
+                mbar_arrive_expect_tx(bar(full0 + st), sbytes);
+                for (int c = 0; c < nch; ++c) tma_load_3d(dst + c * kChunk, &mapRow, bar(full0 + st), 64 * c, w.t * kNk, w.seq);
+                n_loads = n + 1;
                 MLA_TRACE_POINT(0, n);
             }
         }
-    } else if (warp == 1) {
-        // ======================================================== S issuer (whole warp waits, lane 0 issues)
+    } else if (rank == 0 && warp == 1) {
+        // ======================================================== scorer: S issuer (whole warp waits, lane 0 issues)
+        // S(g) = Q-hat . row^T over all 576 columns (36 MMAs of K = 16, Q-hat
+        // from TMEM) into buffer g%2; the stage is released as soon as S(g)
+        // completes.
         constexpr uint32_t idS = idesc_bf16_f32(kHeads, kNk, false, false);
-        const uint32_t stages = base + kOffStages;
-        // Descriptor templates: the start-address field (bits 0..13, address >> 4)
-        // is advanced by adding byte offsets >> 4.
-        const uint64_t dLatK = smem_desc(stages, 16, 1024, kSw128);       // cache latent, K-major (S)
-        const uint64_t dRopeK = smem_desc(stages, 16, 512, kSw64);        // cache RoPE, K-major (S)
-        const uint64_t dQR = smem_desc(base + kOffQR, 16, 512, kSw64);    // Q-hat RoPE half (S, A operand)
-        // S(g) = Q-hat half . cache half^T over this CTA's 288 columns, in tile
-        // order: each S waits for its piece's Q-hat, its tile and S(g-1) to be
-        // read out of TMEM.  (The O MMAs are issued by warp 10: issuing blocks
-        // at the tensor pipe's pace, and a ready O must not wait behind an S.)
+        const uint64_t dRowK = smem_desc(base + kOffSStages, 16, 1024, kSw128);  // cache rows, K-major
         TileWalk ws;
         ws.init(args.plan, grp);
         int T_s = ws.valid ? args.seqlens[ws.seq] : 0;  // length of the sequence of tile g
         bool ok = true;
         for (int g = 0; ws.valid && ok && !*abort_flag; ++g) {
-            if (ws.first() && !MLA_TW(kTwQFull, mbar_wait(bar(kBarQFull), ws.seg & 1))) { ok = false; break; }
-            const uint32_t tile_off = kOffStages + (g % kStages) * kStageBytes;
-            if (!MLA_TW(kTwFull, mbar_wait(bar(kBarFull0 + g % kStages), (g / kStages) & 1))) { ok = false; break; }
-#ifdef MLA_TRACE
-            if (lane == 0) MLA_TRACE_POINT(10, g);
-#endif
-            if (g > 0 && !MLA_TW(kTwSFree, mbar_wait(bar(kBarSFree), (g - 1) & 1))) { ok = false; break; }
+            const int sb = g & 1, st = g % kSStages;
+            if (ws.first() && !MLA_TW(kTwQFull, warp_wait(bar(kBarQFull), ws.seg & 1, lim))) { ok = false; break; }
+            if (!MLA_TW(kTwFull, warp_wait(bar(kBarFull0 + st), (g / kSStages) & 1, lim))) { ok = false; break; }
+            if (g >= 2 && !MLA_TW(kTwSFree, warp_wait(bar(kBarSFree0 + sb), ((g >> 1) - 1) & 1, lim))) { ok = false; break; }
+            const uint32_t tile = base + kOffSStages + st * kSStageBytes;
             const int valid = T_s - ws.t * kNk;
-            if (valid < kNk) {
-                // Rows at or beyond T_b hold no cached token: zero the latent
-                // part so that masked (p = 0) rows cannot inject NaN/Inf into P.C.
-                const int r0 = valid < 0 ? 0 : valid;
-                for (int row = r0 + (lane >> 3); row < kNk; row += 4)
-                    for (int c = 0; c < 4; ++c)
-                        st_shared_v4(base + tile_off + c * kChunk + row * 128 + (lane & 7) * 16, 0, 0, 0, 0);
-                fence_proxy_async_smem();
-            }
+            if (valid < kNk) zero_rows(tile, 9, valid < 0 ? 0 : valid, lane);
             __syncwarp();
             tc_fence_after();
             if (lane == 0) {
                 MLA_TRACE_POINT(14, g);
-#ifdef MLA_TRACE_CYCLES
-                const long long c_s0 = clock64();
-#endif
-                const uint32_t dS = tmem + kTmemS;
-                const uint64_t dL = dLatK + (tile_off >> 4);
+                const uint32_t dS = tmem + kTmemS + 64 * sb;
+                const uint64_t dB = dRowK + ((st * kSStageBytes) >> 4);
 #pragma unroll
-                for (int k = 0; k < 16; ++k)
-                    mma_f16_ts(dS, tmem + kTmemQ + 8 * k, dL + (((k >> 2) * kChunk + 32 * (k & 3)) >> 4), idS,
-                               k ? 1u : 0u);
-#pragma unroll
-                for (int j = 0; j < 2; ++j)
-                    mma_f16_ss(dS, dQR + ((32 * j) >> 4), dRopeK + ((tile_off + 4 * kChunk + 32 * j) >> 4), idS, 1u);
-                mma_commit(bar(kBarSFull));
+                for (int k = 0; k < 36; ++k)
+                    mma_f16_ts(dS, tmem + kTmemQ + 8 * k, dB + (((k >> 2) * kChunk + 32 * (k & 3)) >> 4), idS, k ? 1u : 0u);
+                mma_commit(bar(kBarSFull0 + sb));
+                mma_commit(bar(kBarEmpty0 + st));
+                if (ws.last()) mma_commit(bar(kBarQRead));
                 MLA_TRACE_POINT(1, g);
-                if (g == 0) MLA_TRACE_ALL(2, global_timer_ns());
-#ifdef MLA_TRACE_CYCLES
-                if (cl == MLA_TRACE_CLUSTER && g < kTraceTiles) g_mla_trace[r][g][11] = (unsigned long long)(clock64() - c_s0);
-#endif
             }
             __syncwarp();
             const int seq_before = ws.seq;
@@ -514,71 +521,27 @@ __global__ void __launch_bounds__(kAttThreads, 1)
             if (ws.valid && ws.seq != seq_before) T_s = args.seqlens[ws.seq];
         }
         if (!ok) *abort_flag = 1;
-    } else if (warp == 10) {
-        // ======================================================== O issuer (whole warp waits, lane 0 issues)
-        // O += P(g) . cache latent half(g); the first tile of a piece overwrites
-        // O (after the previous piece's epilogue has read it).
-        constexpr uint32_t idO = idesc_bf16_f32(kHeads, kHalfLat, false, true);
-        const uint64_t dLatMN = smem_desc(base + kOffStages, kChunk, 1024, kSw128);  // cache latent, MN-major
-        TileWalk wo;
-        wo.init(args.plan, grp);
+    } else if (rank == 0 && warp >= 6 && warp <= 9) {
+        // ======================================================== scorer: Q-hat loaders
+        // Row m's 576 Q-hat values -> TMEM columns 0..287 (this thread), once
+        // per piece; the next piece's Q-hat goes in after the last S of the
+        // current piece has completed (S reads Q-hat from TMEM), which the S
+        // issuer signals on its own barrier, one phase per piece: the loaders
+        // are never more than one phase behind it.
         bool ok = true;
-        for (int g = 0; wo.valid && ok && !*abort_flag; ++g, wo.advance()) {
-            if (!MLA_TW(kTwPFull, mbar_wait(bar(kBarPFull0 + (g & 1)), (g >> 1) & 1))) { ok = false; break; }
-            if (wo.first() && wo.seg > 0 && !MLA_TW(kTwOFree, mbar_wait(bar(kBarOFree), (wo.seg - 1) & 1))) { ok = false; break; }
-            tc_fence_after();
-            if (lane == 0) {
-                MLA_TRACE_POINT(15, g);
-                const bool first = wo.first();
-                const int st = g % kStages;
-                const uint64_t dB = dLatMN + ((kOffStages + st * kStageBytes) >> 4);
-                const uint32_t pA = tmem + kTmemP + 32 * (g & 1);
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    mma_f16_ts(tmem + kTmemO, pA + 8 * k, dB + ((2048 * k) >> 4), idO, (!first || k > 0) ? 1u : 0u);
-                mma_commit(bar(kBarPFree0 + (g & 1)));
-                mma_commit(bar(kBarEmpty0 + st));
-                if (wo.last()) mma_commit(bar(kBarOFull));
-                MLA_TRACE_POINT(2, g);
-                MLA_TRACE_ALL(3, global_timer_ns());
-                MLA_TRACE_ALL(6, (unsigned long long)(g + 1));
-                MLA_TRACE_ALL(7, (unsigned long long)(wo.seg + 1));
-            }
-            __syncwarp();
-        }
-        if (!ok) *abort_flag = 1;
-    } else if (warp == 11) {
-        // spare warp (keeps the softmax halves on the same SMSPs as their quarters)
-    } else if (warp >= 6 && warp <= 9) {
-        // ======================================================== exchange warps 6..9
-        const float sl2 = args.scale_log2;
-        const uint32_t x_peer = mapa(base + kOffX, peer);
-        const uint32_t xfull_peer = mapa(bar(kBarXFull0), peer);
-        bool ok = true;
-        // Q-hat of unit u, this CTA's half: row m's 256 latent values -> TMEM
-        // (this thread), the 128 x 32 RoPE block -> shared memory by TMA
-        // (issued by thread 192).
         auto load_q = [&](int u) {
-            if (threadIdx.x == 192) {
-                mbar_arrive_expect_tx(bar(kBarQFull), kQRBytes);
-                tma_load_3d(base + kOffQR, &mapQR, bar(kBarQFull), kLat + kHalfRope * r, 0, u);
-            }
-            const uint4* src = reinterpret_cast<const uint4*>(args.q_hat + ((size_t)u * kHeads + m) * kRow) + 32 * r;
+            const uint4* src = reinterpret_cast<const uint4*>(args.q_hat + ((size_t)u * kHeads + m) * kRow);
+#pragma unroll 1
+            for (int c = 0; c < 9; ++c) {
+                uint4 x[8];
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint4 x[16];
+                for (int j = 0; j < 8; ++j) x[j] = __ldg(src + 8 * c + j);
+                uint32_t v[32];
 #pragma unroll
-                for (int j = 0; j < 16; ++j) x[j] = __ldg(src + 16 * half + j);
-#pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    uint32_t v[32];
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        v[4 * j] = x[8 * c + j].x; v[4 * j + 1] = x[8 * c + j].y;
-                        v[4 * j + 2] = x[8 * c + j].z; v[4 * j + 3] = x[8 * c + j].w;
-                    }
-                    tmem_st32(tmem + lane_addr + kTmemQ + 64 * half + 32 * c, v);
+                for (int j = 0; j < 8; ++j) {
+                    v[4 * j] = x[j].x; v[4 * j + 1] = x[j].y; v[4 * j + 2] = x[j].z; v[4 * j + 3] = x[j].w;
                 }
+                tmem_st32(tmem + lane_addr + kTmemQ + 32 * c, v);
             }
             tmem_wait_st();
             tc_fence_before();
@@ -588,116 +551,59 @@ __global__ void __launch_bounds__(kAttThreads, 1)
         TileWalk w;
         w.init(args.plan, grp);
         if (w.valid) load_q(w.seq * q_len + qi);
-        if (threadIdx.x == 192) MLA_TRACE_POINT(3, kTraceProlog);
-        for (int h = 0; w.valid && ok && !*abort_flag; ++h, w.advance()) {
-            const int hb = h & 1;
-            // ---- partial S(h) of this half, in log2 units, rounded to fp16
-            if (!MLA_TW(kTwSFull, mbar_wait(bar(kBarSFull), h & 1))) { ok = false; break; }
+        for (; w.valid && ok && !*abort_flag; w.advance()) {
+            if (!w.last()) continue;
+            TileWalk nx = w;
+            nx.advance();
+            if (!nx.valid) break;
+            // every S of piece w.seg has read Q-hat
+            if (!warp_wait(bar(kBarQRead), w.seg & 1, lim)) { ok = false; break; }
             tc_fence_after();
-            uint32_t own[32];
-            {
-                // both halves out of TMEM first, so that S(h+1) may start at once
-                uint32_t va[32], vb[32];
-                tmem_ld32(tmem + lane_addr + kTmemS, va);
-                tmem_ld32(tmem + lane_addr + kTmemS + 32, vb);
-                tmem_wait_ld();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(kBarSFree));
-#pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    own[j] = pack_f16(__uint_as_float(va[2 * j]) * sl2, __uint_as_float(va[2 * j + 1]) * sl2);
-                    own[16 + j] = pack_f16(__uint_as_float(vb[2 * j]) * sl2, __uint_as_float(vb[2 * j + 1]) * sl2);
-                }
-                if (threadIdx.x == 192) MLA_TRACE_POINT(3, h);
-            }
-            // ---- publish: Own[hb] (read by our softmax warps and by the bulk copy
-            // into the peer's X[hb]); both readers of tile h-2 must be done.
-            if (h >= 2) {
-                if (!MLA_TW(kTwOwnFree, mbar_wait(bar(kBarOwnFree0 + hb), ((h >> 1) - 1) & 1))) { ok = false; break; }
-                if (!MLA_TW(kTwOwnFree, mbar_wait_cluster(bar(kBarXFree0 + hb), ((h >> 1) - 1) & 1))) { ok = false; break; }
-            }
-            const uint32_t own_buf = base + kOffOwn + hb * kXBytes;
-#pragma unroll
-            for (int c = 0; c < 8; ++c)
-                st_shared_v4(own_buf + sw128(m, c), own[4 * c], own[4 * c + 1], own[4 * c + 2], own[4 * c + 3]);
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-                const uint32_t off = quarter * 32 * 128;
-                bulk_copy_s2s(x_peer + hb * kXBytes + off, own_buf + off, 32 * 128, xfull_peer + 8 * hb);
-                mbar_arrive(bar(kBarOwnFull0 + hb));
-            }
-            // The peer's partial for tile h lands in our X[hb] (its phase h/2).
-            if (threadIdx.x == 192) {
-                mbar_arrive_expect_tx(bar(kBarXFull0 + hb), kXBytes);
-                MLA_TRACE_POINT(4, h);
-            }
-            // S(h) was the last reader of this piece's Q-hat: load the next
-            // piece's, after the partial is on its way (the next S waits for it,
-            // the exchange of tile h does not).
-            if (w.last()) {
-                TileWalk nx = w;
-                nx.advance();
-                if (nx.valid) load_q(nx.seq * q_len + qi);
-            }
+            load_q(nx.seq * q_len + qi);
         }
         if (!ok) *abort_flag = 1;
-    } else {
-        // ======================================================== softmax warps 2..5 and 12..15
+    } else if (rank == 0 && softmax_warp) {
+        // ======================================================== scorer: softmax warps 2..5 and 12..15
         // Two warps per TMEM quarter: half kh takes keys 32kh..32kh+31 of each
-        // score row and latent columns 128kh..128kh+127 of O; the pair agrees on
-        // the row maximum through shared memory, meeting on named barrier
-        // 1 + quarter.  Both warps walk the same tiles and meet at the same
-        // points; a failed (timed-out) wait does not leave the loop at once: the
-        // warp skips the tile's side effects up to the next meeting, where both
-        // read each other's status and stop together (a hardware barrier has no
-        // time limit, so neither may wait at one the other never reaches).
-        const int kh = warp >= 12 ? 1 : 0;
-        const uint32_t xfree_peer = mapa(bar(kBarXFree0), peer);
+        // score row; the pair agrees on the row maximum through shared memory,
+        // meeting on named barrier 1 + quarter.  Both warps walk the same tiles
+        // and meet at the same points; a failed (timed-out) wait does not leave
+        // the loop at once: the warp skips the tile's side effects up to the
+        // next meeting, where both read each other's status and stop together.
+        // P goes to the accumulator's slot g % kPSlots with st.async (SW128
+        // rows, the O MMA's A operand), with this row's rescale factor of O
+        // and the half's running sum of p.
+        const uint32_t pslot_peer = mapa(base + kOffPSlots, peer);
+        const uint32_t pfull_peer = mapa(bar(kBarPFull0), peer);
         float* red = reinterpret_cast<float*>(base_ptr + kOffRed);  // [2 tiles][2 halves][128 rows]
         volatile int* pair_ok = reinterpret_cast<volatile int*>(base_ptr + kOffFlags);
+        const float sl2 = args.scale_log2;
         bool ok = true;
         TileWalk w;
         w.init(args.plan, grp);
         float m_used = -CUDART_INF_F, l_part = 0.f;
         int n_keys = 0;
         for (int g = 0; w.valid; ++g, w.advance()) {
-            const int b2 = g & 1;
-            // ---- S(g) for this thread's 32 keys = own partial + the peer's (same order on both CTAs)
-            if (ok) ok = MLA_TW(kTwXFull, mbar_wait(bar(kBarOwnFull0 + b2), (g >> 1) & 1));
-            if (ok) ok = MLA_TW(kTwXFull, mbar_wait_cluster(bar(kBarXFull0 + b2), (g >> 1) & 1));
+            const int sb = g & 1, b2 = g & 1, slot = g % kPSlots;
+            if (ok) ok = MLA_TW(kTwXFull, warp_wait(bar(kBarSFull0 + sb), (g >> 1) & 1, lim));
             float s[32];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) s[j] = 0.f;
             if (ok) {
-                const uint32_t own_buf = base + kOffOwn + b2 * kXBytes;
-                const uint32_t x_buf = base + kOffX + b2 * kXBytes;
+                tc_fence_after();
+                uint32_t v[32];
+                tmem_ld32(tmem + lane_addr + kTmemS + 64 * sb + 32 * kh, v);
+                tmem_wait_ld();
 #pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
-                    const int c = 4 * kh + cc;
-                    uint32_t a0, a1, a2, a3, o0, o1, o2, o3;
-                    ld_shared_v4u(own_buf + sw128(m, c), a0, a1, a2, a3);
-                    ld_shared_v4u(x_buf + sw128(m, c), o0, o1, o2, o3);
-                    const uint32_t mine[4] = {a0, a1, a2, a3};
-                    const uint32_t oth[4] = {o0, o1, o2, o3};
+                for (int j = 0; j < 32; ++j) s[j] = __uint_as_float(v[j]) * sl2;
+            } else {
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const float2 v = sum_f16x2(mine[q], oth[q]);
-                        s[8 * cc + 2 * q] = v.x;
-                        s[8 * cc + 2 * q + 1] = v.y;
-                    }
-                }
+                for (int j = 0; j < 32; ++j) s[j] = 0.f;
             }
-            // Both buffers are consumed (their values are in registers and used
-            // by the adds above), so relaxed arrives suffice.
+            tc_fence_before();
             __syncwarp();
-            if (ok && lane == 0) {
-                mbar_arrive(bar(kBarOwnFree0 + b2));
-                mbar_arrive_remote_relaxed(xfree_peer + 8 * b2);
-            }
-            if (threadIdx.x == 64) MLA_TRACE_POINT(5, g);
-            // ---- online softmax in base 2, lazy rescaling of O
+            if (ok && lane == 0) mbar_arrive(bar(kBarSFree0 + sb));
+            if (threadIdx.x == 64) MLA_TRACE_POINT(3, g);
+            // ---- online softmax in base 2; O (in the accumulator) is rescaled
+            // lazily, only when the row maximum grows by more than 2^8.
             // query token qi of sequence b sees keys 0..T_b-q_len+qi
             if (w.first()) n_keys = args.seqlens[w.seq] - q_len + 1 + qi;
             const int key0 = w.t * kNk + 32 * kh;
@@ -722,11 +628,17 @@ __global__ void __launch_bounds__(kAttThreads, 1)
                 break;
             }
             const float mx = fmaxf(rg[m], rg[kHeads + m]);
-            if (threadIdx.x == 64) MLA_TRACE_POINT(8, g);
             const bool first = w.first();
-            const bool grow = mx > m_used + 8.0f;  // rescale only when the max grows by > 2^8
-            const float mb_new = grow ? mx : m_used;
-            const float mb = (mb_new == -CUDART_INF_F) ? 0.f : mb_new;
+            const bool grow = mx > m_used + 8.0f;
+            float f = 1.0f;  // factor the accumulator applies to O's row before adding P(g)
+            if (grow) {
+                if (!first) {
+                    f = ex2(m_used - mx);
+                    l_part *= f;
+                }
+                m_used = mx;
+            }
+            const float mb = (m_used == -CUDART_INF_F) ? 0.f : m_used;
             uint32_t pk[16];
             float rs0 = 0.f, rs1 = 0.f;
 #pragma unroll
@@ -736,117 +648,220 @@ __global__ void __launch_bounds__(kAttThreads, 1)
                 rs1 += p1;
                 pk[j] = pack_bf16(p0, p1);
             }
-            if (threadIdx.x == 64) MLA_TRACE_POINT(9, g);
-            // P buffer b2 was last read by O(g-2).  (From here to the next
-            // meeting a failed wait only skips work.)
-            if (g >= 2 && ok) ok = MLA_TW(kTwPFree, mbar_wait(bar(kBarPFree0 + b2), ((g >> 1) - 1) & 1));
-            if (grow && ok) {
-                if (!first) {
-                    // O must hold everything up to tile g-1 before it is rescaled.
-                    ok = MLA_TW(kTwPFree, mbar_wait(bar(kBarPFree0 + (b2 ^ 1)), ((g - 1) >> 1) & 1));
-                }
-                if (ok && !first) {
-                    tc_fence_after();
-                    const float f = ex2(m_used - mx);
-                    l_part *= f;
-#pragma unroll 1
-                    for (int c0 = 0; c0 < kHalfLat / 2; c0 += 32) {
-                        uint32_t v[32];
-                        tmem_ld32(tmem + lane_addr + kTmemO + 128 * kh + c0, v);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * f);
-                        tmem_st32(tmem + lane_addr + kTmemO + 128 * kh + c0, v);
-                    }
-                }
-                m_used = mx;
-            }
+            l_part += rs0 + rs1;
+            // ---- send P(g): the accumulator must have consumed slot g%kPSlots
+            // (tile g - kPSlots), which also means the bulk copies that read
+            // the local staging slot have completed.  Each warp writes its half
+            // rows into the staging slot; once both halves of the quarter are
+            // in, one lane copies the quarter's rows (4 KB of P, 512 bytes of
+            // row data) to the peer.
+            // (from here to the next meeting a failed wait only skips work)
+            if (ok && g >= kPSlots)
+                ok = MLA_TW(kTwPFree, warp_wait_cluster(bar(kBarSlotFree0 + slot), ((g / kPSlots) - 1) & 1, lim));
+            const uint32_t stg = base + kOffStaging + slot * kPSlotBytes;
             if (ok) {
-                tc_fence_after();
-                l_part += rs0 + rs1;
-                tmem_st16(tmem + lane_addr + kTmemP + 32 * b2 + 16 * kh, pk);
-                tmem_wait_st();
-                tc_fence_before();
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc)
+                    st_shared_v4(stg + sw128(m, 4 * kh + cc), pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
+                // row data: {f, l_part of half 0} from half 0, {l_part of half 1, 0} from half 1
+                st_shared_v2(stg + kPData + 16 * m + 8 * kh, kh ? __float_as_uint(l_part) : __float_as_uint(f),
+                             kh ? 0u : __float_as_uint(l_part));
+                fence_proxy_async_smem();
             }
-            __syncwarp();
-            if (ok && lane == 0) mbar_arrive(bar(kBarPFull0 + b2));
-            if (threadIdx.x == 64) MLA_TRACE_POINT(6, g);
-#ifndef MLA_TRACE_CYCLES
-            if (threadIdx.x == 96) MLA_TRACE_POINT(11, g);
-            if (threadIdx.x == 384) MLA_TRACE_POINT(12, g);
-#endif
-            if (threadIdx.x == 160) MLA_TRACE_POINT(13, g);
-            // ---- epilogue at the end of a piece: this thread owns O row m, columns 128kh..+127
-            float l_sum = 0.f;
+            volatile int* wr_pair = pair_ok + 16 + (b2 * 4 + quarter) * 2;  // this tile's "written" status
+            if (lane == 0) wr_pair[kh] = ok ? 1 : 0;
+            named_bar_sync(1 + quarter, 64);
+            if (kh == 0) {
+                const bool both = wr_pair[0] && wr_pair[1];
+                if (both && lane == 0) {
+                    const uint32_t dst = pslot_peer + slot * kPSlotBytes;
+                    const uint32_t pb = pfull_peer + 8 * slot;
+                    bulk_copy_s2s(dst + quarter * 4096, stg + quarter * 4096, 4096, pb);
+                    bulk_copy_s2s(dst + kPData + quarter * 512, stg + kPData + quarter * 512, 512, pb);
+                }
+                if (!both) ok = false;
+            }
+            if (threadIdx.x == 64) MLA_TRACE_POINT(4, g);
+            // ---- end of a piece: the LSE of a split piece (base 2), from both halves' sums
             if (w.last()) {
-                // the row's softmax denominator: both halves' partial sums
                 float* rl = red + (b2 * 2) * kHeads;
                 named_bar_sync(1 + quarter, 64);  // the pair has read this tile's maxima
                 rl[kh * kHeads + m] = l_part;
                 named_bar_sync(1 + quarter, 64);
-                l_sum = rl[m] + rl[kHeads + m];
-                if (ok) ok = mbar_wait(bar(kBarOFull), w.seg & 1);
-            }
-            if (w.last() && ok) {
-                tc_fence_after();
-                const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
-                const int u = w.seq * q_len + qi;
-                const int col0 = r * kHalfLat + 128 * kh;  // first latent column of this thread
-                if (w.whole) {
-                    __nv_bfloat16* dst = args.o_lat + ((size_t)u * kHeads + m) * kLat + col0;
-#pragma unroll 1
-                    for (int c0 = 0; c0 < kHalfLat / 2; c0 += 32) {
-                        uint32_t v[32];
-                        tmem_ld32(tmem + lane_addr + kTmemO + 128 * kh + c0, v);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int j = 0; j < 32; j += 16) {
-                            uint32_t o[8];
-#pragma unroll
-                            for (int q = 0; q < 8; ++q)
-                                o[q] = pack_bf16(__uint_as_float(v[j + 2 * q]) * inv, __uint_as_float(v[j + 2 * q + 1]) * inv);
-                            if (args.o_lat_v8) {
-                                st_global_v8(dst + c0 + j, o[0], o[1], o[2], o[3], o[4], o[5], o[6], o[7]);
-                            } else {
-                                *reinterpret_cast<uint4*>(dst + c0 + j) = make_uint4(o[0], o[1], o[2], o[3]);
-                                *reinterpret_cast<uint4*>(dst + c0 + j + 8) = make_uint4(o[4], o[5], o[6], o[7]);
-                            }
-                        }
-                    }
-                } else {
-                    // fp32 partial in column octets, [slot][c8][head][8]: a warp (32
-                    // consecutive heads) writes 1 KB contiguous per octet (one 32-byte
-                    // store per lane), and a consumer reading one head gets whole
-                    // 32-byte sectors.
-                    const size_t slot = (size_t)(grp + w.seq) * q_len + qi;
-                    float* dst = args.part_o + (slot * (kLat / 8) * kHeads + m) * 8;
-#pragma unroll 1
-                    for (int c0 = 0; c0 < kHalfLat / 2; c0 += 32) {
-                        uint32_t v[32];
-                        tmem_ld32(tmem + lane_addr + kTmemO + 128 * kh + c0, v);
-                        tmem_wait_ld();
-                        const int o0 = (col0 + c0) / 8;
-#pragma unroll
-                        for (int j = 0; j < 32; j += 8) {
-                            uint32_t o[8];
-#pragma unroll
-                            for (int q = 0; q < 8; ++q) o[q] = __float_as_uint(__uint_as_float(v[j + q]) * inv);
-                            st_global_v8(dst + (size_t)(o0 + j / 8) * kHeads * 8, o[0], o[1], o[2], o[3], o[4], o[5],
-                                         o[6], o[7]);
-                        }
-                    }
-                    if (r == 0 && kh == 0)
-                        args.part_lse[slot * kHeads + m] = l_sum > 0.f ? m_used + __log2f(l_sum) : -CUDART_INF_F;
+                const float l_sum = rl[m] + rl[kHeads + m];
+                if (ok && !w.whole && kh == 0) {
+                    const size_t pslot = (size_t)(grp + w.seq) * q_len + qi;
+                    args.part_lse[pslot * kHeads + m] = l_sum > 0.f ? m_used + __log2f(l_sum) : -CUDART_INF_F;
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(kBarOFree));
-                if (threadIdx.x == 64) MLA_TRACE_POINT(7, g);
-                if (threadIdx.x == 64) MLA_TRACE_POINT(5, kTraceProlog);
-                if (threadIdx.x == 64) MLA_TRACE_ALL(4, global_timer_ns());
                 m_used = -CUDART_INF_F;
                 l_part = 0.f;
             }
+        }
+        if (!ok) *abort_flag = 1;
+    } else if (rank == 1 && warp == 1) {
+        // ======================================================== accumulator: O issuer (whole warp waits, lane 0 issues)
+        // O += P(g) . latent(g) (N = 512 as two MMAs of N = 256 per K step,
+        // P from the slot, the latent MN-major from the stage); the first tile
+        // of a piece overwrites O after the previous piece's epilogue read it.
+        constexpr uint32_t idO = idesc_bf16_f32(kHeads, 256, false, true);
+        const uint64_t dP = smem_desc(base + kOffPSlots, 16, 1024, kSw128);          // P, K-major
+        const uint64_t dV = smem_desc(base + kOffVStages, kChunk, 1024, kSw128);     // latent, MN-major
+        TileWalk wo;
+        wo.init(args.plan, grp);
+        int T_o = wo.valid ? args.seqlens[wo.seq] : 0;
+        bool ok = true;
+        for (int g = 0; wo.valid && ok && !*abort_flag; ++g) {
+            const int slot = g % kPSlots, st = g % kVStages;
+            const uint32_t ph = (g / kPSlots) & 1;
+            if (!MLA_TW(kTwPFull, warp_wait_cluster(bar(kBarPFull0 + slot), ph, lim))) { ok = false; break; }
+            if (!MLA_TW(kTwPFull, warp_wait(bar(kBarRescaled0 + slot), ph, lim))) { ok = false; break; }
+            if (!MLA_TW(kTwFull, warp_wait(bar(kBarVFull0 + st), (g / kVStages) & 1, lim))) { ok = false; break; }
+            if (wo.first() && wo.seg > 0 &&
+                !MLA_TW(kTwOFree, warp_wait(bar(kBarOFree), (wo.seg - 1) & 1, lim))) { ok = false; break; }
+            const uint32_t tile = base + kOffVStages + st * kVStageBytes;
+            const int valid = T_o - wo.t * kNk;
+            if (valid < kNk) zero_rows(tile, 8, valid < 0 ? 0 : valid, lane);
+            __syncwarp();
+            tc_fence_after();
+            if (lane == 0) {
+                MLA_TRACE_POINT(15, g);
+                const bool first = wo.first();
+                const uint64_t a0 = dP + ((slot * kPSlotBytes) >> 4);
+                const uint64_t b0 = dV + ((st * kVStageBytes) >> 4);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+#pragma unroll
+                    for (int hf = 0; hf < 2; ++hf)
+                        mma_f16_ss(tmem + kTmemO + 256 * hf, a0 + ((32 * k) >> 4), b0 + ((4 * kChunk * hf + 2048 * k) >> 4),
+                                   idO, (!first || k > 0) ? 1u : 0u);
+                mma_commit(bar(kBarPDone0 + slot));
+                mma_commit(bar(kBarVEmpty0 + st));
+                if (wo.last()) mma_commit(bar(kBarOFull));
+                MLA_TRACE_POINT(2, g);
+            }
+            __syncwarp();
+            const int seq_before = wo.seq;
+            wo.advance();
+            if (wo.valid && wo.seq != seq_before) T_o = args.seqlens[wo.seq];
+        }
+        if (!ok) *abort_flag = 1;
+    } else if (rank == 1 && warp == 10) {
+        // ======================================================== accumulator: slot forwarder (lane 0)
+        // Arms each P slot for the scorer's next tile in it (expected bytes),
+        // then tells the scorer the slot is free, once the O MMA that read it
+        // has completed.
+        TileWalk w;
+        w.init(args.plan, grp);
+        int n_tiles = 0;
+        for (TileWalk c = w; c.valid; c.advance()) ++n_tiles;
+        const uint32_t slotfree_peer = mapa(bar(kBarSlotFree0), peer);
+        bool ok = true;
+        if (lane == 0)
+            for (int s = 0; s < kPSlots && s < n_tiles; ++s) mbar_arrive_expect_tx(bar(kBarPFull0 + s), kPSlotBytes);
+        for (int g = 0; g + kPSlots < n_tiles && ok && !*abort_flag; ++g) {
+            const int slot = g % kPSlots;
+            if (!warp_wait(bar(kBarPDone0 + slot), (g / kPSlots) & 1, lim)) { ok = false; break; }
+            if (lane == 0) {
+                mbar_arrive_expect_tx(bar(kBarPFull0 + slot), kPSlotBytes);  // for tile g + kPSlots
+                mbar_arrive_remote_relaxed(slotfree_peer + 8 * slot);
+            }
+        }
+        if (!ok) *abort_flag = 1;
+    } else if (rank == 1 && softmax_warp) {
+        // ======================================================== accumulator: rescale / epilogue warps
+        // Two warps per TMEM quarter: half kh owns O columns 256kh..256kh+255
+        // of its rows.  Per tile: apply the scorer's rescale factor to O rows
+        // whose maximum grew (the whole warp, factor 1 on the other rows),
+        // then release the O MMA; at the end of a piece, normalise O and store
+        // o_lat (bf16) or the split partial (fp32).
+        const float* slots = reinterpret_cast<const float*>(base_ptr + kOffPSlots);
+        bool ok = true;
+        TileWalk w;
+        w.init(args.plan, grp);
+        for (int g = 0; w.valid && ok && !*abort_flag; ++g, w.advance()) {
+            const int slot = g % kPSlots;
+            if (!MLA_TW(kTwXFull, warp_wait_cluster(bar(kBarPFull0 + slot), (g / kPSlots) & 1, lim))) { ok = false; break; }
+            // the row data {f, l of half 0, l of half 1, 0}: read before the slot
+            // is released (the scorer refills it once O(g) has completed)
+            const float* rowdat = slots + (slot * kPSlotBytes + kPData) / 4 + 4 * m;
+            const float f = rowdat[0];
+            const float l_sum = rowdat[1] + rowdat[2];
+            const bool first = w.first();
+            if (!first && __any_sync(0xffffffffu, f != 1.0f)) {
+                // O must hold everything up to tile g-1 before it is rescaled
+                const int ps = (g - 1) % kPSlots;
+                if (!warp_wait(bar(kBarPDone0 + ps), ((g - 1) / kPSlots) & 1, lim)) { ok = false; break; }
+                tc_fence_after();
+#pragma unroll 1
+                for (int c0 = 0; c0 < 256; c0 += 32) {
+                    uint32_t v[32];
+                    tmem_ld32(tmem + lane_addr + kTmemO + 256 * kh + c0, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * f);
+                    tmem_st32(tmem + lane_addr + kTmemO + 256 * kh + c0, v);
+                }
+                tmem_wait_st();
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(kBarRescaled0 + slot));
+            if (threadIdx.x == 64) MLA_TRACE_POINT(5, g);
+            if (!w.last()) continue;
+            // ---- epilogue: this thread owns O row m, columns 256kh..256kh+255
+            if (!warp_wait(bar(kBarOFull), w.seg & 1, lim)) { ok = false; break; }
+            tc_fence_after();
+            const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
+            const int u = w.seq * q_len + qi;
+            const int col0 = 256 * kh;
+            if (w.whole) {
+                __nv_bfloat16* dst = args.o_lat + ((size_t)u * kHeads + m) * kLat + col0;
+#pragma unroll 1
+                for (int c0 = 0; c0 < 256; c0 += 32) {
+                    uint32_t v[32];
+                    tmem_ld32(tmem + lane_addr + kTmemO + col0 + c0, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 32; j += 16) {
+                        uint32_t o[8];
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            o[q] = pack_bf16(__uint_as_float(v[j + 2 * q]) * inv, __uint_as_float(v[j + 2 * q + 1]) * inv);
+                        if (args.o_lat_v8) {
+                            st_global_v8(dst + c0 + j, o[0], o[1], o[2], o[3], o[4], o[5], o[6], o[7]);
+                        } else {
+                            *reinterpret_cast<uint4*>(dst + c0 + j) = make_uint4(o[0], o[1], o[2], o[3]);
+                            *reinterpret_cast<uint4*>(dst + c0 + j + 8) = make_uint4(o[4], o[5], o[6], o[7]);
+                        }
+                    }
+                }
+            } else {
+                // fp32 partial in column octets, [slot][c8][head][8]: a warp (32
+                // consecutive heads) writes 1 KB contiguous per octet (one 32-byte
+                // store per lane), and a consumer reading one head gets whole
+                // 32-byte sectors.
+                const size_t pslot = (size_t)(grp + w.seq) * q_len + qi;
+                float* dst = args.part_o + (pslot * (kLat / 8) * kHeads + m) * 8;
+#pragma unroll 1
+                for (int c0 = 0; c0 < 256; c0 += 32) {
+                    uint32_t v[32];
+                    tmem_ld32(tmem + lane_addr + kTmemO + col0 + c0, v);
+                    tmem_wait_ld();
+                    const int o0 = (col0 + c0) / 8;
+#pragma unroll
+                    for (int j = 0; j < 32; j += 8) {
+                        uint32_t o[8];
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) o[q] = __float_as_uint(__uint_as_float(v[j + q]) * inv);
+                        st_global_v8(dst + (size_t)(o0 + j / 8) * kHeads * 8, o[0], o[1], o[2], o[3], o[4], o[5], o[6],
+                                     o[7]);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(kBarOFree));
+            if (threadIdx.x == 64) MLA_TRACE_POINT(7, g);
         }
         if (!ok) *abort_flag = 1;
     }
@@ -858,15 +873,36 @@ __global__ void __launch_bounds__(kAttThreads, 1)
             if (tw_acc[i]) MLA_TRACE_ALL(kTwBase + i, tw_acc[i]);
     }
 #endif
-    if (*abort_flag && threadIdx.x == 0) atomicOr(args.status, MLA_STATUS_TIMEOUT);
+    // ---- teardown: nothing this CTA issued may still be running when it exits.
+    // On normal completion every stage load, MMA and incoming P slot was
+    // waited for by its consumer.  After an expired wait the roles stopped
+    // early, so what they had issued is drained here (each wait again bounded).
+    __syncthreads();  // every role has stopped issuing; the abort flag is final
+    const bool aborted = *abort_flag != 0;
+    if (aborted && active && warp == 0 && lane == 0) {  // stage loads in flight
+        const int nst = rank == 0 ? kSStages : kVStages;
+        const int full0 = rank == 0 ? kBarFull0 : kBarVFull0;
+        for (int n = n_loads > nst ? n_loads - nst : 0; n < n_loads; ++n)
+            mbar_wait(bar(full0 + n % nst), (n / nst) & 1, lim);
+    }
+    // Every MMA of the issuer (a commit tracks all prior MMAs of its thread).
+    if (warp == 1 && lane == 0) mma_commit(bar(kBarDrain));
+    if (warp == 1) mbar_wait(bar(kBarDrain), 0, lim);
+    if (aborted && threadIdx.x == 0) atomicOr(args.status, MLA_STATUS_TIMEOUT);
     tc_fence_before();
     __syncthreads();
     if (warp == 1) tmem_dealloc(tmem, kTmemCols);
-    // The peer may still copy scores into this CTA's shared memory or arrive
-    // on its barriers: neither CTA leaves before both are done.
     if (threadIdx.x == 0) MLA_TRACE_POINT(6, kTraceProlog);
+    // The peer may still arrive on this CTA's barriers: neither CTA leaves
+    // before both have stopped.  P rows the scorer stored into the
+    // accumulator's shared memory with st.async are not ordered by the
+    // cluster barrier; they have all landed unless a CTA stopped early, in
+    // which case both give them time to land before the shared memory is
+    // released.
     cluster_sync();
-    if (threadIdx.x == 0) MLA_TRACE_POINT(7, kTraceProlog);
+    const bool peer_aborted = ld_shared_cluster_u32(mapa(abort_addr, peer)) != 0;
+    cluster_sync();
+    if (aborted || peer_aborted) spin_ns(20000);
     if (threadIdx.x == 0) MLA_TRACE_ALL(5, global_timer_ns());
     MLA_KT(kKtAttend, 2);
 }

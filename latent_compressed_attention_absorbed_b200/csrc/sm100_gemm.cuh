@@ -201,7 +201,8 @@ __global__ void __launch_bounds__(128, 1)
     }
 
     // ---------------- epilogue: all four warps, TMEM lane quarter = warp
-    const bool ok = mbar_wait(done_bar, 0) && !*abort_flag;
+    // warp-uniform: the TMEM loads below are whole-warp (.aligned) instructions
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(done_bar, 0) && !*abort_flag);
     tc_fence_after();
     const int row = m0 + warp * 32 + lane;
     if (ok) {

@@ -40,7 +40,7 @@ def test_library_exports_every_declared_symbol(built):
 def test_library_loads_and_reports_version(built):
     from latent_compressed_attention_absorbed_b200 import binding
     lib = binding.Library(built)
-    assert lib.version() == 100
+    assert lib.version() == 101
     assert lib.lib.mla_last_error() == b""
 
 
