@@ -349,7 +349,69 @@ def run_ours(args, rank, world, local_rank):
         e2e = {"value": round(e2e_ms * 1e3, 3), "unit": "us/step", "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h), "timing": "host wall clock per step incl. synchronize"}
     times = {"ms_step": ms_step, "ms_med": ms_med, "ms_warm": ms_warm, "ms_append": ms_append}
-    return cfg, path, times, stage_ms, clk.summary(), e2e
+    proj = None if args.no_projections or path != "sm100" else time_projections(
+        torch, lib, dims, cfg, device, out, flush, args.steps)
+    return cfg, path, times, stage_ms, clk.summary(), e2e, proj
+
+
+def time_projections(torch, lib, dims, cfg, device, attn_out, flush, steps):
+    """The projections around the decode at this step's rows (B * q_len tokens):
+    the cache append from the block input x and the output projection W_O,
+    each a CUDA graph replayed with L2 flushed between replays."""
+    rows = cfg.B * cfg.q_len
+    x = upload(torch, wl.block_input(cfg, cfg.q_len), device)
+    w_a, gamma = wl.append_weights(cfg)
+    W_A, g = upload(torch, w_a, device), upload(torch, gamma, device)
+    W_O = upload(torch, wl.output_weights(cfg), device)
+    del w_a, gamma
+    scratch = torch.zeros((cfg.B, cfg.q_len, cfg.row), dtype=W_A.dtype, device=device)
+    pos0 = torch.zeros(cfg.B, dtype=torch.int32, device=device)
+    y = torch.empty((rows, cfg.d_model), dtype=W_O.dtype, device=device)
+    ws_a = torch.empty(lib.lib.mla_append_from_hidden_workspace_bytes(dims, cfg.B, cfg.q_len, cfg.d_model),
+                       dtype=torch.uint8, device=device)
+    ws_o = torch.empty(lib.lib.mla_output_projection_workspace_bytes(dims, rows, cfg.d_model), dtype=torch.uint8,
+                       device=device)
+    calls = {
+        "append_from_hidden": lambda st: lib.append_from_hidden(dims, scratch, x, W_A, g, pos0, workspace=ws_a,
+                                                                stream=st),
+        "output_projection": lambda st: lib.output_projection(dims, attn_out, W_O, y=y, workspace=ws_o, stream=st),
+    }
+    es = 2
+    nbytes = {
+        "append_from_hidden": (cfg.row * cfg.d_model + rows * cfg.d_model + rows * cfg.row + cfg.d_c) * es,
+        "output_projection": (cfg.d_model * cfg.H * cfg.d_v + rows * cfg.H * cfg.d_v + rows * cfg.d_model) * es,
+    }
+    pk, _ = peaks()
+    res = {}
+    stream = torch.cuda.current_stream()
+    for name, call in calls.items():
+        s = torch.cuda.Stream(device)
+        s.wait_stream(stream)
+        with torch.cuda.stream(s):
+            call(s)
+        stream.wait_stream(s)
+        torch.cuda.synchronize()
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=s):
+            call(s)
+        torch.cuda.synchronize()
+        ev = []
+        for _ in range(max(20, min(steps, 200))):
+            torch.cuda._sleep(100000)
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            gr.replay()
+            b.record(stream)
+            ev.append((a, b))
+        torch.cuda.synchronize()
+        us = float(np.mean([a.elapsed_time(b) for a, b in ev])) * 1e3
+        gbps = nbytes[name] / (us * 1e-6) / 1e9
+        res[name] = {"us": round(us, 3), "algorithmic_bytes": int(nbytes[name]), "gbps": round(gbps, 1),
+                     "frac_of_hbm": round(gbps / pk["hbm_gbs"], 4), "rows": rows, "d_model": cfg.d_model}
+        del gr
+    assert lib.device_status() == 0
+    return res
 
 
 class OracleSample:
@@ -436,6 +498,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-projections", action="store_true", help="skip timing the projections around the decode")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--ref-budget", type=float, default=5.0, help="seconds of oracle work per reference step")
     args = ap.parse_args()
@@ -456,7 +519,7 @@ def main():
         torch.cuda.set_device(local_rank)
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local_rank))
-    cfg, path, times, stage_ms, clocks, e2e = run_ours(args, rank, world, local_rank)
+    cfg, path, times, stage_ms, clocks, e2e, proj = run_ours(args, rank, world, local_rank)
     ms_step, ms_med = times["ms_step"], times["ms_med"]
     if world > 1:
         import torch
@@ -530,6 +593,8 @@ def main():
         "clocks": clocks,
         "e2e": e2e,
     }
+    if proj:
+        line["projections"] = proj
     if args.gpus == 1 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg, args.cpu_budget)
     print(json.dumps(line), flush=True)
