@@ -80,22 +80,24 @@ constexpr int kRow = kLat + kRope;
 //   red, flags: the softmax pairs' row maxima / sums and their status.
 // Accumulating CTA (cluster rank 1):
 //   vstages: kVStages latent parts of 64 keys (8 SW128 chunks), 64 KB each;
-//   pslots:  kPSlots slots, each P of 128 heads x 64 keys (bf16, SW128,
-//            K-major: the A operand of the O MMA) followed by 16 bytes per
-//            head: the rescale factor of O and the two halves' sums of p.
+//   pslots:  kPSlots slots, each P of 128 heads x 64 keys as two matrices of
+//            32 keys (bf16, 64-byte rows, SW64, K-major: the A operand of the
+//            O MMA's first and last two K steps), then per key half and head
+//            8 bytes: the rescale factor of O and that half's sum of p.
 constexpr int kChunk = kNk * 128;            // 8192: 64 keys x 64 columns
 constexpr int kSStages = 2;
 constexpr int kSStageBytes = 9 * kChunk;     // 73728
 constexpr int kVStages = 2;
 constexpr int kVStageBytes = 8 * kChunk;     // 65536
 constexpr int kPSlots = 3;
-constexpr int kPData = kHeads * 128;         // 16384
-constexpr int kPSlotBytes = kPData + kHeads * 16;  // 18432
+constexpr int kPHalf = kHeads * 64;          // 8192: one key half of P
+constexpr int kPData = 2 * kPHalf;           // 16384
+constexpr int kPSlotBytes = kPData + 2 * kHeads * 8;  // 18432
 constexpr int kOffSStages = 0;
 constexpr int kOffStaging = kSStages * kSStageBytes;
 constexpr int kOffRed = kOffStaging + kPSlots * kPSlotBytes;  // [2 tiles][2 halves][128 rows] fp32
-constexpr int kOffFlags = kOffRed + 2 * 2 * kHeads * 4;       // [2 tiles][4 quarters][2] int, twice
-constexpr int kScorerEnd = kOffFlags + 2 * 2 * 4 * 2 * 4;
+constexpr int kOffFlags = kOffRed + 2 * 2 * kHeads * 4;       // [2 tiles][4 quarters][2] int
+constexpr int kScorerEnd = kOffFlags + 2 * 4 * 2 * 4;
 #ifndef MLA_SCORE_PREFETCH
 #define MLA_SCORE_PREFETCH 0
 #endif
@@ -331,6 +333,8 @@ struct AttendArgs {
 // reads (K-major, 1024-byte groups of 8 rows), and the 8 rows a quarter-warp
 // touches at once land in 8 different bank groups.
 __device__ __forceinline__ uint32_t sw128(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
+// The same for 64-byte rows (SW64: chunk c of row r moves to c ^ ((r / 2) % 4)).
+__device__ __forceinline__ uint32_t sw64(int r, int c) { return (uint32_t)(r * 64 + ((c ^ ((r >> 1) & 3)) << 4)); }
 
 // Rows at or beyond the sequence length hold no cached token: zero `nchunks`
 // SW128 chunks of 64 keys from row r0 on (one warp), so that masked rows can
@@ -651,35 +655,27 @@ __global__ void __launch_bounds__(kAttThreads, 1)
             l_part += rs0 + rs1;
             // ---- send P(g): the accumulator must have consumed slot g%kPSlots
             // (tile g - kPSlots), which also means the bulk copies that read
-            // the local staging slot have completed.  Each warp writes its half
-            // rows into the staging slot; once both halves of the quarter are
-            // in, one lane copies the quarter's rows (4 KB of P, 512 bytes of
-            // row data) to the peer.
+            // the local staging slot have completed.  This warp's half rows
+            // are a contiguous 2 KB of its key half's matrix (and 256 bytes
+            // of row data), so it copies them to the peer itself.
             // (from here to the next meeting a failed wait only skips work)
             if (ok && g >= kPSlots)
                 ok = MLA_TW(kTwPFree, warp_wait_cluster(bar(kBarSlotFree0 + slot), ((g / kPSlots) - 1) & 1, lim));
-            const uint32_t stg = base + kOffStaging + slot * kPSlotBytes;
             if (ok) {
+                const uint32_t stg = base + kOffStaging + slot * kPSlotBytes;
 #pragma unroll
                 for (int cc = 0; cc < 4; ++cc)
-                    st_shared_v4(stg + sw128(m, 4 * kh + cc), pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
-                // row data: {f, l_part of half 0} from half 0, {l_part of half 1, 0} from half 1
-                st_shared_v2(stg + kPData + 16 * m + 8 * kh, kh ? __float_as_uint(l_part) : __float_as_uint(f),
-                             kh ? 0u : __float_as_uint(l_part));
+                    st_shared_v4(stg + kPHalf * kh + sw64(m, cc), pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
+                st_shared_v2(stg + kPData + 1024 * kh + 8 * m, __float_as_uint(f), __float_as_uint(l_part));
                 fence_proxy_async_smem();
-            }
-            volatile int* wr_pair = pair_ok + 16 + (b2 * 4 + quarter) * 2;  // this tile's "written" status
-            if (lane == 0) wr_pair[kh] = ok ? 1 : 0;
-            named_bar_sync(1 + quarter, 64);
-            if (kh == 0) {
-                const bool both = wr_pair[0] && wr_pair[1];
-                if (both && lane == 0) {
+                __syncwarp();
+                if (lane == 0) {
                     const uint32_t dst = pslot_peer + slot * kPSlotBytes;
                     const uint32_t pb = pfull_peer + 8 * slot;
-                    bulk_copy_s2s(dst + quarter * 4096, stg + quarter * 4096, 4096, pb);
-                    bulk_copy_s2s(dst + kPData + quarter * 512, stg + kPData + quarter * 512, 512, pb);
+                    const uint32_t po = kPHalf * kh + quarter * 32 * 64, ao = kPData + 1024 * kh + quarter * 32 * 8;
+                    bulk_copy_s2s(dst + po, stg + po, 32 * 64, pb);
+                    bulk_copy_s2s(dst + ao, stg + ao, 32 * 8, pb);
                 }
-                if (!both) ok = false;
             }
             if (threadIdx.x == 64) MLA_TRACE_POINT(4, g);
             // ---- end of a piece: the LSE of a split piece (base 2), from both halves' sums
@@ -704,7 +700,7 @@ __global__ void __launch_bounds__(kAttThreads, 1)
         // P from the slot, the latent MN-major from the stage); the first tile
         // of a piece overwrites O after the previous piece's epilogue read it.
         constexpr uint32_t idO = idesc_bf16_f32(kHeads, 256, false, true);
-        const uint64_t dP = smem_desc(base + kOffPSlots, 16, 1024, kSw128);          // P, K-major
+        const uint64_t dP = smem_desc(base + kOffPSlots, 16, 512, kSw64);            // P key halves, K-major
         const uint64_t dV = smem_desc(base + kOffVStages, kChunk, 1024, kSw128);     // latent, MN-major
         TileWalk wo;
         wo.init(args.plan, grp);
@@ -732,8 +728,8 @@ __global__ void __launch_bounds__(kAttThreads, 1)
                 for (int k = 0; k < 4; ++k)
 #pragma unroll
                     for (int hf = 0; hf < 2; ++hf)
-                        mma_f16_ss(tmem + kTmemO + 256 * hf, a0 + ((32 * k) >> 4), b0 + ((4 * kChunk * hf + 2048 * k) >> 4),
-                                   idO, (!first || k > 0) ? 1u : 0u);
+                        mma_f16_ss(tmem + kTmemO + 256 * hf, a0 + ((kPHalf * (k >> 1) + 32 * (k & 1)) >> 4),
+                                   b0 + ((4 * kChunk * hf + 2048 * k) >> 4), idO, (!first || k > 0) ? 1u : 0u);
                 mma_commit(bar(kBarPDone0 + slot));
                 mma_commit(bar(kBarVEmpty0 + st));
                 if (wo.last()) mma_commit(bar(kBarOFull));
@@ -781,11 +777,12 @@ __global__ void __launch_bounds__(kAttThreads, 1)
         for (int g = 0; w.valid && ok && !*abort_flag; ++g, w.advance()) {
             const int slot = g % kPSlots;
             if (!MLA_TW(kTwXFull, warp_wait_cluster(bar(kBarPFull0 + slot), (g / kPSlots) & 1, lim))) { ok = false; break; }
-            // the row data {f, l of half 0, l of half 1, 0}: read before the slot
-            // is released (the scorer refills it once O(g) has completed)
-            const float* rowdat = slots + (slot * kPSlotBytes + kPData) / 4 + 4 * m;
+            // the row data {f, this half's sum of p} of both key halves: read
+            // before the slot is released (the scorer refills it once O(g) has
+            // completed)
+            const float* rowdat = slots + (slot * kPSlotBytes + kPData) / 4 + 2 * m;
             const float f = rowdat[0];
-            const float l_sum = rowdat[1] + rowdat[2];
+            const float l_sum = rowdat[1] + rowdat[1024 / 4 + 1];
             const bool first = w.first();
             if (!first && __any_sync(0xffffffffu, f != 1.0f)) {
                 // O must hold everything up to tile g-1 before it is rescaled
