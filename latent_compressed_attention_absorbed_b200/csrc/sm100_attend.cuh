@@ -77,7 +77,9 @@ constexpr int kRow = kLat + kRope;
 //            x 64 columns (latent 0..511, then RoPE 512..575), 72 KB each;
 //   staging: kPSlots local copies of the accumulator's P slots (same layout),
 //            written by the softmax warps and bulk-copied to the peer;
-//   red, flags: the softmax pairs' row maxima / sums and their status.
+//   red, flags: the softmax pairs' row maxima / sums and their status;
+//   qstage:  per TMEM quarter, one 128-byte column block of its 32 Q-hat rows
+//            (the Q-hat loaders read rows coalesced and transpose them here).
 // Accumulating CTA (cluster rank 1):
 //   vstages: kVStages latent parts of 64 keys (8 SW128 chunks), 64 KB each;
 //   pslots:  kPSlots slots, each P of 128 heads x 64 keys as two matrices of
@@ -97,7 +99,8 @@ constexpr int kOffSStages = 0;
 constexpr int kOffStaging = kSStages * kSStageBytes;
 constexpr int kOffRed = kOffStaging + kPSlots * kPSlotBytes;  // [2 tiles][2 halves][128 rows] fp32
 constexpr int kOffFlags = kOffRed + 2 * 2 * kHeads * 4;       // [2 tiles][4 quarters][2] int
-constexpr int kScorerEnd = kOffFlags + 2 * 4 * 2 * 4;
+constexpr int kOffQStage = (kOffFlags + 2 * 4 * 2 * 4 + 127) & ~127;  // [4 quarters][32 rows][128 B]: Q-hat transpose
+constexpr int kScorerEnd = kOffQStage + 4 * 32 * 128;
 #ifndef MLA_SCORE_PREFETCH
 #define MLA_SCORE_PREFETCH 0
 #endif
@@ -147,8 +150,10 @@ static_assert(8 * (kNumBars + 2) <= kBarBytes, "barrier block too small");
 
 // Optional timing trace (compile with -DMLA_TRACE): global-timer stamps (ns)
 // of both CTAs of one cluster at fixed points of every tile, read back by
-// mla_trace_read.  Scorer: 0 stage loads issued, 14 S issue start, 1 S
-// issued, 3 S read by the softmax warps, 4 P handed to the bulk copies.
+// mla_trace_read.  Scorer: 0 stage loads issued, 6 stage landed (seen by
+// the S issuer), 14 S issue start, 1 S issued, 12 S complete (seen by a
+// softmax warp), 3 / 13 S read by the two softmax warps of quarter 2, 8 row
+// maximum agreed, 9 P computed, 10 slot free, 4 P handed to the bulk copies.
 // Accumulator: 0 stage loads issued, 5 O rows rescaled (or checked), 15 O
 // issue start, 2 O issued, 7 piece epilogue done.
 #ifdef MLA_TRACE
@@ -501,6 +506,7 @@ __global__ void __launch_bounds__(kAttThreads, 1)
             const int sb = g & 1, st = g % kSStages;
             if (ws.first() && !MLA_TW(kTwQFull, warp_wait(bar(kBarQFull), ws.seg & 1, lim))) { ok = false; break; }
             if (!MLA_TW(kTwFull, warp_wait(bar(kBarFull0 + st), (g / kSStages) & 1, lim))) { ok = false; break; }
+            if (lane == 0) MLA_TRACE_POINT(6, g);
             if (g >= 2 && !MLA_TW(kTwSFree, warp_wait(bar(kBarSFree0 + sb), ((g >> 1) - 1) & 1, lim))) { ok = false; break; }
             const uint32_t tile = base + kOffSStages + st * kSStageBytes;
             const int valid = T_s - ws.t * kNk;
@@ -533,19 +539,43 @@ __global__ void __launch_bounds__(kAttThreads, 1)
         // issuer signals on its own barrier, one phase per piece: the loaders
         // are never more than one phase behind it.
         bool ok = true;
+        // Rows are read coalesced (a warp instruction covers four whole 128-byte
+        // row blocks), staged in shared memory with the 16-byte pieces of row r
+        // permuted by r % 8, and read back one row per lane for tcgen05.st;
+        // the next column block's loads are in flight during the transpose.
+        const uint32_t qbuf = base + kOffQStage + quarter * 32 * 128;
+        const int rr = lane >> 3, pc = lane & 7;  // this lane's row within a group of four, and 16-byte piece
         auto load_q = [&](int u) {
-            const uint4* src = reinterpret_cast<const uint4*>(args.q_hat + ((size_t)u * kHeads + m) * kRow);
+            const uint4* src = reinterpret_cast<const uint4*>(args.q_hat + ((size_t)u * kHeads + quarter * 32) * kRow);
+            uint4 cur[8], nxt[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) cur[j] = __ldg(src + (size_t)(4 * j + rr) * (kRow / 8) + pc);
 #pragma unroll 1
             for (int c = 0; c < 9; ++c) {
-                uint4 x[8];
+                if (c + 1 < 9) {
 #pragma unroll
-                for (int j = 0; j < 8; ++j) x[j] = __ldg(src + 8 * c + j);
-                uint32_t v[32];
+                    for (int j = 0; j < 8; ++j) nxt[j] = __ldg(src + (size_t)(4 * j + rr) * (kRow / 8) + 8 * (c + 1) + pc);
+                }
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
-                    v[4 * j] = x[j].x; v[4 * j + 1] = x[j].y; v[4 * j + 2] = x[j].z; v[4 * j + 3] = x[j].w;
+                    const int row = 4 * j + rr;
+                    st_shared_v4(qbuf + row * 128 + ((pc ^ (row & 7)) << 4), cur[j].x, cur[j].y, cur[j].z, cur[j].w);
                 }
-                tmem_st32(tmem + lane_addr + kTmemQ + 32 * c, v);
+                __syncwarp();
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t v[16];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int piece = 4 * h + q;
+                        ld_shared_v4u(qbuf + lane * 128 + ((piece ^ (lane & 7)) << 4), v[4 * q], v[4 * q + 1], v[4 * q + 2],
+                                      v[4 * q + 3]);
+                    }
+                    tmem_st16(tmem + lane_addr + kTmemQ + 32 * c + 16 * h, v);
+                }
+                __syncwarp();  // the buffer is rewritten for the next block
+#pragma unroll
+                for (int j = 0; j < 8; ++j) cur[j] = nxt[j];
             }
             tmem_wait_st();
             tc_fence_before();
@@ -590,6 +620,7 @@ __global__ void __launch_bounds__(kAttThreads, 1)
         for (int g = 0; w.valid; ++g, w.advance()) {
             const int sb = g & 1, b2 = g & 1, slot = g % kPSlots;
             if (ok) ok = MLA_TW(kTwXFull, warp_wait(bar(kBarSFull0 + sb), (g >> 1) & 1, lim));
+            if (threadIdx.x == 64) MLA_TRACE_POINT(12, g);
             float s[32];
             if (ok) {
                 tc_fence_after();
@@ -606,6 +637,7 @@ __global__ void __launch_bounds__(kAttThreads, 1)
             __syncwarp();
             if (ok && lane == 0) mbar_arrive(bar(kBarSFree0 + sb));
             if (threadIdx.x == 64) MLA_TRACE_POINT(3, g);
+            if (threadIdx.x == 448) MLA_TRACE_POINT(13, g);
             // ---- online softmax in base 2; O (in the accumulator) is rescaled
             // lazily, only when the row maximum grows by more than 2^8.
             // query token qi of sequence b sees keys 0..T_b-q_len+qi
@@ -632,6 +664,7 @@ __global__ void __launch_bounds__(kAttThreads, 1)
                 break;
             }
             const float mx = fmaxf(rg[m], rg[kHeads + m]);
+            if (threadIdx.x == 64) MLA_TRACE_POINT(8, g);
             const bool first = w.first();
             const bool grow = mx > m_used + 8.0f;
             float f = 1.0f;  // factor the accumulator applies to O's row before adding P(g)
@@ -653,6 +686,7 @@ __global__ void __launch_bounds__(kAttThreads, 1)
                 pk[j] = pack_bf16(p0, p1);
             }
             l_part += rs0 + rs1;
+            if (threadIdx.x == 64) MLA_TRACE_POINT(9, g);
             // ---- send P(g): the accumulator must have consumed slot g%kPSlots
             // (tile g - kPSlots), which also means the bulk copies that read
             // the local staging slot have completed.  This warp's half rows
@@ -661,6 +695,7 @@ __global__ void __launch_bounds__(kAttThreads, 1)
             // (from here to the next meeting a failed wait only skips work)
             if (ok && g >= kPSlots)
                 ok = MLA_TW(kTwPFree, warp_wait_cluster(bar(kBarSlotFree0 + slot), ((g / kPSlots) - 1) & 1, lim));
+            if (threadIdx.x == 64) MLA_TRACE_POINT(10, g);
             if (ok) {
                 const uint32_t stg = base + kOffStaging + slot * kPSlotBytes;
 #pragma unroll
