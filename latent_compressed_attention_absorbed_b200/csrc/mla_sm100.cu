@@ -201,14 +201,24 @@ static cudaError_t absorb_gemv_launch(const AbsorbGemvArgs& a, cudaStream_t st) 
     constexpr int idx = R == 1 ? 0 : R == 2 ? 1 : R == 4 ? 2 : 3;
     cudaError_t e = set_smem(absorb_gemv_kernel<R>, absorb_gemv_smem<R>(), g_smem_absorb_gemv[idx]);
     if (e != cudaSuccess) return e;
-    return launch_pdl(absorb_gemv_kernel<R>, dim3(kHeads + 1, 2), dim3(128), absorb_gemv_smem<R>(), st, 1, a);
+    // W_UK [128 heads][128][512]: one box of 256 latent columns x 128 rows per CTA
+    CUtensorMap mapW;
+    if (!make_map(&mapW, a.W_UK, kLat, 128, kHeads, (uint64_t)kLat * 2, (uint64_t)128 * kLat * 2, 256, 128, 1,
+                  CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    return launch_pdl(absorb_gemv_kernel<R>, dim3(kHeads + 1, 2), dim3(128), absorb_gemv_smem<R>(), st, 1, mapW, a);
 }
 template <int R>
 static cudaError_t project_gemv_launch(const ProjectGemvArgs& a, cudaStream_t st) {
     constexpr int idx = R == 1 ? 0 : R == 2 ? 1 : R == 4 ? 2 : 3;
     cudaError_t e = set_smem(project_gemv_kernel<R>, project_gemv_smem<R>(), g_smem_project_gemv[idx]);
     if (e != cudaSuccess) return e;
-    return launch_pdl(project_gemv_kernel<R>, dim3(kHeads), dim3(512), project_gemv_smem<R>(), st, 1, a);
+    // W_UV [128 heads][128][512]: eight SW128 boxes of 64 latent columns x 128 rows per CTA
+    CUtensorMap mapW;
+    if (!make_map(&mapW, a.W_UV, kLat, 128, kHeads, (uint64_t)kLat * 2, (uint64_t)128 * kLat * 2, 64, 128, 1,
+                  CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    return launch_pdl(project_gemv_kernel<R>, dim3(kHeads), dim3(512), project_gemv_smem<R>(), st, 1, mapW, a);
 }
 
 cudaError_t sm100_absorb_small(const Problem& p, const void* q_nope, const void* q_rope, const void* W_UK,
@@ -347,6 +357,7 @@ cudaError_t sm100_project_small(const Problem& p, void* attend_workspace, int nu
     a.W_UV = (const __nv_bfloat16*)W_UV;
     a.rows = rows;
     a.out = (__nv_bfloat16*)out;
+    a.status = device_status_ptr();
     if (rows == 1) return project_gemv_launch<1>(a, st);
     if (rows == 2) return project_gemv_launch<2>(a, st);
     if (rows <= 4) return project_gemv_launch<4>(a, st);

@@ -9,8 +9,9 @@
 // (092 page, section 二 "缓存压缩也可以做一个代数检查": fold U^T into the query
 // once; ailearn.mscapital.top MLA panel: W_UV after the latent aggregation.)
 //
-// Each CTA stages its 64 KB slice of the weights in shared memory with
-// cp.async before waiting for the previous kernel (weights are never
+// Each CTA stages its slice of the weights in shared memory with TMA (one
+// 64 KB box for absorb, eight 16 KB boxes for project, all completing on one
+// mbarrier) before waiting for the previous kernel (weights are never
 // written by it), so the weight stream overlaps the previous kernel's tail.
 // The project kernel also merges the split-KV partials of the attention
 // step itself (so the decode needs no separate combine launch for these
@@ -29,19 +30,18 @@ namespace sm100 {
 
 constexpr int kGemvMaxRows = 8;
 constexpr int kGemvWBytes = 64 * 1024;  // weight slice of one CTA
-template <int R> constexpr int absorb_gemv_smem() { return kGemvWBytes + R * 128 * 4; }
+// + the mbarrier (16 bytes) and slack to align the TMA destination to 128 bytes
+template <int R> constexpr int absorb_gemv_smem() { return kGemvWBytes + R * 128 * 4 + 16 + 128; }
 constexpr int kMergeStateFloats = kLat + 4;  // acc[512], m, wsum (padded)
 constexpr int kProjWarps = 16;                 // project CTA: 512 threads, all 128 output rows of a head
-constexpr int kProjWRow = kLat * 2 + 16;       // W_UV row in shared memory, padded: lanes hit distinct banks
-constexpr int kProjWBytes = 128 * kProjWRow;   // W_UV[h]: 130 KB
+// W_UV[h] in shared memory: eight SW128 boxes of 64 latent columns x 128 rows
+// (row v's 16-byte chunk c of box k at k*16 KB + v*128 + ((c ^ (v % 8)) * 16),
+// so the eight rows a quarter-warp reads at once hit distinct banks)
+constexpr int kProjWBytes = 128 * kLat * 2;    // 128 KB
 template <int R> constexpr int project_gemv_smem() {
-    return kProjWBytes + R * kLat * 4 + kProjWarps * kMergeStateFloats * 4 + 4 * R * 128 * 4;
+    return kProjWBytes + R * kLat * 4 + kProjWarps * kMergeStateFloats * 4 + 4 * R * 128 * 4 + 16 + 1024;
 }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 __device__ __forceinline__ float2 bf16x2_to_f2(uint32_t v) {
     return make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u));
@@ -65,11 +65,15 @@ struct AbsorbGemvArgs {
 // grid (129, 2), 128 threads: CTA (h, y) produces latent columns
 // 256y..256y+255 of head h for every row and RoPE pairs 16y..16y+15; CTA
 // (128, 0) writes the attention plan.  Thread t owns columns 2t, 2t+1.
+// mapW: W_UK as [128 heads][128 d][512 c] bf16, box 256 c x 128 d, no swizzle
+// (the box lands as w_s[d][256]).
 template <int R>
-__global__ void __launch_bounds__(128) absorb_gemv_kernel(AbsorbGemvArgs a) {
-    extern __shared__ __align__(16) uint8_t gemv_smem[];
+__global__ void __launch_bounds__(128) absorb_gemv_kernel(const __grid_constant__ CUtensorMap mapW, AbsorbGemvArgs a) {
+    extern __shared__ __align__(16) uint8_t gemv_smem_raw[];
+    uint8_t* gemv_smem = gemv_smem_raw + ((128u - (smem_u32(gemv_smem_raw) & 127u)) & 127u);
     auto w_s = reinterpret_cast<__nv_bfloat16(*)[256]>(gemv_smem);                 // W_UK[h][d][256y ..]
     auto q_s = reinterpret_cast<float(*)[128]>(gemv_smem + kGemvWBytes);          // q_nope rows, fp32
+    const uint32_t wbar = smem_u32(gemv_smem + kGemvWBytes + R * 128 * 4);
     const int h = blockIdx.x, y = blockIdx.y, t = threadIdx.x;
     MLA_KT(kKtAbsorb, 0);
     if (h == kHeads) {
@@ -81,15 +85,12 @@ __global__ void __launch_bounds__(128) absorb_gemv_kernel(AbsorbGemvArgs a) {
         MLA_KT(kKtAbsorb, 2);
         return;
     }
-    // weights first (they do not depend on the previous kernel): 128 rows x 512 B
-    {
-        const uint32_t ws = smem_u32(&w_s[0][0]);
-        const __nv_bfloat16* src = a.W_UK + (size_t)h * 128 * kLat + 256 * y;
-#pragma unroll 4
-        for (int i = t; i < 128 * 32; i += 128) {
-            const int d = i / 32, c = i % 32;
-            cp_async16(ws + d * 512 + c * 16, src + (size_t)d * kLat + c * 8);
-        }
+    // weights first (they do not depend on the previous kernel): one 64 KB box
+    if (t == 0) {
+        mbar_init(wbar, 1);
+        fence_mbar_init();
+        mbar_arrive_expect_tx(wbar, kGemvWBytes);
+        tma_load_3d(smem_u32(&w_s[0][0]), &mapW, wbar, 256 * y, 0, h);
     }
     pdl_wait();
     if (t == 0) pdl_trigger();
@@ -112,8 +113,12 @@ __global__ void __launch_bounds__(128) absorb_gemv_kernel(AbsorbGemvArgs a) {
                 __floats2bfloat162_rn(y0, y1);
         }
     }
-    cp_async_wait_all();
-    __syncthreads();
+    __syncthreads();  // q_s, and the barrier's initialisation, are visible to every thread
+    if (!mbar_wait(wbar, 0, MLA_WAIT_LIMIT_NS)) {
+        atomicOr(a.status, MLA_STATUS_TIMEOUT);
+        mbar_wait(wbar, 0, MLA_WAIT_LIMIT_NS);  // the copy must not land after the CTA has exited
+        return;
+    }
     float acc[R][2];
 #pragma unroll
     for (int u = 0; u < R; ++u) acc[u][0] = acc[u][1] = 0.f;
@@ -144,6 +149,7 @@ struct ProjectGemvArgs {
     const __nv_bfloat16* W_UV;    // [128][128][512]
     int rows;
     __nv_bfloat16* out;           // [rows][128][128]
+    int* status;
 };
 
 // grid (128), 512 threads: CTA h produces all 128 output columns of head h.
@@ -155,11 +161,13 @@ struct ProjectGemvArgs {
 //   2. thread (v, q) forms the dot products of output row v with every row
 //      over latent columns 128q..128q+127; the four partial sums are added
 //      through shared memory.
+// mapW: W_UV as [128 heads][128 v][512 c] bf16, box 64 c x 128 v, SW128.
 template <int R>
-__global__ void __launch_bounds__(512) project_gemv_kernel(ProjectGemvArgs a) {
+__global__ void __launch_bounds__(512) project_gemv_kernel(const __grid_constant__ CUtensorMap mapW, ProjectGemvArgs a) {
     constexpr int G = kProjWarps / R;
-    extern __shared__ __align__(16) uint8_t gemv_smem[];
-    uint8_t* w_s = gemv_smem;                                                          // W_UV[h][v][:], padded rows
+    extern __shared__ __align__(16) uint8_t gemv_smem_raw[];
+    uint8_t* gemv_smem = gemv_smem_raw + ((1024u - (smem_u32(gemv_smem_raw) & 1023u)) & 1023u);
+    uint8_t* w_s = gemv_smem;                                                          // W_UV[h], eight SW128 boxes
     auto o_s = reinterpret_cast<float(*)[kLat]>(gemv_smem + kProjWBytes);              // o_lat rows, fp32
     auto st_s = reinterpret_cast<float(*)[kMergeStateFloats]>(gemv_smem + kProjWBytes + R * kLat * 4);
     auto sum_s = reinterpret_cast<float(*)[R][128]>(gemv_smem + kProjWBytes + R * kLat * 4 +
@@ -168,14 +176,14 @@ __global__ void __launch_bounds__(512) project_gemv_kernel(ProjectGemvArgs a) {
     const int warp = t / 32, lane = t % 32;
     const int u = warp % R, g = warp / R;
     MLA_KT(kKtProject, 0);
-    {
-        const uint32_t ws = smem_u32(w_s);
-        const __nv_bfloat16* src = a.W_UV + (size_t)h * 128 * kLat;
-#pragma unroll 4
-        for (int i = t; i < 128 * 64; i += 512) {
-            const int v = i / 64, c = i % 64;  // row v, 16-byte chunk c
-            cp_async16(ws + v * kProjWRow + c * 16, src + (size_t)v * kLat + c * 8);
-        }
+    const uint32_t wbar = smem_u32(gemv_smem + kProjWBytes + R * kLat * 4 + kProjWarps * kMergeStateFloats * 4 +
+                                   4 * R * 128 * 4);
+    if (t == 0) {
+        mbar_init(wbar, 1);
+        fence_mbar_init();
+        mbar_arrive_expect_tx(wbar, kProjWBytes);
+#pragma unroll 1
+        for (int k = 0; k < 8; ++k) tma_load_3d(smem_u32(w_s) + k * 16384, &mapW, wbar, 64 * k, 0, h);
     }
     pdl_wait();
     if (t == 0) pdl_trigger();
@@ -230,20 +238,21 @@ __global__ void __launch_bounds__(512) project_gemv_kernel(ProjectGemvArgs a) {
             reinterpret_cast<float4*>(&o_s[u][0])[lane + 32 * j] = make_float4(lo.x, lo.y, hi.x, hi.y);
         }
     }
-    cp_async_wait_all();
-    __syncthreads();
+    __syncthreads();  // o_s, and the barrier's initialisation, are visible to every thread
+    const bool w_ok = mbar_wait(wbar, 0, MLA_WAIT_LIMIT_NS);
     // ---- 2. out[u][h][v] = sum_c W_UV[h][v][c] o[u][c]: thread (v, quarter q) takes
-    // output row v = t % 128 and latent columns 128q..128q+127 for every row u;
-    // the four quarters are added through shared memory.
+    // output row v = t % 128 and latent columns 128q..128q+127 (boxes 2q, 2q+1)
+    // for every row u; the four quarters are added through shared memory.
     {
         const int v = t % 128, q = t / 128;
         float acc[R];
 #pragma unroll
         for (int uu = 0; uu < R; ++uu) acc[uu] = 0.f;
-        const uint8_t* wrow = w_s + v * kProjWRow + q * 256;
+        const uint8_t* wrow = w_s + 2 * q * 16384 + v * 128;
 #pragma unroll 2
-        for (int c8 = 0; c8 < 16; ++c8) {
-            const uint4 w8 = *reinterpret_cast<const uint4*>(wrow + c8 * 16);
+        for (int c8 = 0; c8 < 16 && w_ok; ++c8) {
+            const uint4 w8 =
+                *reinterpret_cast<const uint4*>(wrow + (c8 >> 3) * 16384 + (((c8 & 7) ^ (v & 7)) << 4));
             const float2 w01 = bf16x2_to_f2(w8.x), w23 = bf16x2_to_f2(w8.y);
             const float2 w45 = bf16x2_to_f2(w8.z), w67 = bf16x2_to_f2(w8.w);
 #pragma unroll
@@ -267,6 +276,10 @@ __global__ void __launch_bounds__(512) project_gemv_kernel(ProjectGemvArgs a) {
         if (uu < a.rows)
             a.out[((size_t)uu * kHeads + h) * 128 + v] =
                 __float2bfloat16_rn(sum_s[0][uu][v] + sum_s[1][uu][v] + sum_s[2][uu][v] + sum_s[3][uu][v]);
+    }
+    if (!w_ok && t == 0) {
+        atomicOr(a.status, MLA_STATUS_TIMEOUT);
+        mbar_wait(wbar, 0, MLA_WAIT_LIMIT_NS);  // the copies must not land after the CTA has exited
     }
     MLA_KT(kKtProject, 2);
 }
