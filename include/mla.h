@@ -130,7 +130,8 @@ int mla_decode(const mla_dims_t* dims, const void* q_nope, const void* q_rope,
  *         CUDA kernels otherwise), 1 = force the tensor-core path
  *         (MLA_ERR_UNSUPPORTED if it cannot run), 2 = force the generic path.
  *   num_pairs: CTA pairs (clusters) of the attention grid (0 = one per two SMs;
- *         at most 1024).
+ *         larger values are capped to that, the clusters that fit on the
+ *         device at once, for which mla_workspace_bytes() sizes the scratch).
  *   overhead_tiles: scheduling cost charged per query token (each of the
  *         B * q_len tokens is scheduled on its own), in 64-key tiles
  *         (negative = default, 2).

@@ -108,7 +108,10 @@ int choose_path(const Problem& p, int q_len, const mla_decode_opts_t* o, bool* f
 }
 
 int pairs_for(const mla_decode_opts_t* o) {
-    int n = (o && o->num_pairs > 0) ? o->num_pairs : sm100_default_pairs();
+    // At most the clusters that fit on the device at once: more would only
+    // run in a second wave, and mla_workspace_bytes() sizes for that many.
+    const int cap = sm100_default_pairs();
+    int n = (o && o->num_pairs > 0 && o->num_pairs < cap) ? o->num_pairs : cap;
     if (n > 1024) n = 1024;  // the split combine handles at most 1024 pieces per sequence
     return n > 0 ? n : 1;
 }
