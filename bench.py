@@ -76,12 +76,17 @@ def peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+# The sources that define the attention kernel and its launch (grid, plan,
+# workspace): a DRAM capture stays valid while none of them changes.
+ATTEND_SOURCES = ("mla_api.cu", "mla_internal.h", "mla_rope.cuh", "mla_sm100.cu", "sm100_attend.cuh", "sm100_host.h",
+                  "sm100_ptx.cuh")
+
+
 def csrc_hash():
     h = hashlib.sha256()
-    for f in sorted(os.listdir(CSRC)):
-        if f.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(CSRC, f), "rb") as fh:
-                h.update(f.encode() + fh.read())
+    for f in ATTEND_SOURCES:
+        with open(os.path.join(CSRC, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
 
 

@@ -131,7 +131,8 @@ __global__ void __launch_bounds__(128, 1)
         // early stop) would leave their stage waiting for bytes: none can
         // exist, since the loop issues the A half of every pre-issued stage
         // before it can stop (a stop happens only at i >= pre).
-    } else if (warp == 1 && lane == 0) {
+    }
+    if (warp == 1 && lane == 0) {
         // ---------------- MMA issuer
         for (int i = 0; i < nk; ++i) {
             const int s = i % STAGES;
@@ -150,6 +151,10 @@ __global__ void __launch_bounds__(128, 1)
         }
         mma_commit(done_bar);
     }
+    // The other lanes of the producer and MMA warps wait here for their lane 0
+    // (a warp barrier: they must not spin on the completion barrier below
+    // while lane 0 of the same warp runs its loop).
+    __syncwarp();
     pdl_wait();  // nothing is written before the kernels this one depends on have completed
     // ---------------- epilogue: all four warps, TMEM lane quarter = warp
     const bool ok = __all_sync(0xffffffffu, mbar_wait(done_bar, 0, lim) && !*abort_flag) && nk > 0;
