@@ -82,6 +82,21 @@ ATTEND_SOURCES = ("mla_api.cu", "mla_internal.h", "mla_rope.cuh", "mla_sm100.cu"
                   "sm100_ptx.cuh")
 
 
+def replica_config(base, rank):
+    """The workload one rank decodes: same shape, its own seeded sequences."""
+    return base.with_(seed=base.seed + 1000 * rank)
+
+
+def max_over_ranks(values, world, device):
+    """Element-wise maximum of per-rank timings over all ranks (unchanged for one rank)."""
+    if world <= 1:
+        return [float(v) for v in values]
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(x) for x in t]
+
+
 def csrc_hash():
     h = hashlib.sha256()
     for f in ATTEND_SOURCES:
@@ -191,7 +206,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(device)
     lib = binding.load()
     base = wl.CONFIGS[args.workload]
-    cfg = base.with_(seed=base.seed + 1000 * rank)  # each replica decodes its own sequences
+    cfg = replica_config(base, rank)  # each replica decodes its own sequences
     dt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
     dims = lib.dims(cfg.H, cfg.d_c, cfg.d_r, cfg.d_n, cfg.d_v, dt, cfg.rope_base)
 
@@ -297,10 +312,7 @@ def run_ours(args, rank, world, local_rank):
         torch.distributed.barrier()
     ms_step = float(np.mean(times_ms))
     ms_med = float(np.median(times_ms))
-    if world > 1:
-        t = torch.tensor([ms_step, ms_med, ms_warm, ms_append], dtype=torch.float64, device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_step, ms_med, ms_warm, ms_append = (float(x) for x in t)
+    ms_step, ms_med, ms_warm, ms_append = max_over_ranks([ms_step, ms_med, ms_warm, ms_append], world, device)
 
     # ---- per-kernel stage times (same kernels, launched directly with stage events)
     n_ev = binding.NUM_EVENTS
@@ -345,10 +357,7 @@ def run_ours(args, rank, world, local_rank):
             e2e_step()
             wall.append((time.perf_counter() - t0) * 1e3)
         e2e_ms = float(np.mean(wall))
-        if world > 1:
-            t = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            e2e_ms = float(t[0])
+        e2e_ms = max_over_ranks([e2e_ms], world, device)[0]
         h2d = sum(x.numel() * x.element_size() for x in (h_qn, h_qr))
         d2h = h_out.numel() * h_out.element_size()
         e2e = {"value": round(e2e_ms * 1e3, 3), "unit": "us/step", "h2d_bytes_per_step": int(h2d),
