@@ -137,7 +137,15 @@ class Library:
 
     @staticmethod
     def cache_desc(cache: torch.Tensor) -> Cache:
-        _need(cache, "cache", ndim=3)
+        """[B][T_max][row] with unit stride along the row; the other two strides
+        are passed on (a view of a larger buffer: padded rows, or a subset of a
+        larger batch), and the library checks them."""
+        if not cache.is_cuda:
+            raise ValueError("cache must be a CUDA tensor")
+        if cache.dim() != 3:
+            raise ValueError(f"cache must have 3 dims, got {tuple(cache.shape)}")
+        if cache.stride(2) != 1:
+            raise ValueError("cache rows must be contiguous (unit stride along the last dimension)")
         return Cache(cache.data_ptr(), cache.shape[0], cache.shape[1], cache.stride(0), cache.stride(1))
 
     @staticmethod

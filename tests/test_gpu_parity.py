@@ -183,6 +183,28 @@ def test_rope_base_through_append_and_decode(lib, base):
     check_close(as_f64(out), P.oracle_expanded(range(cfg.B)), "bf16", f"rope_base={base}")
 
 
+@pytest.mark.parametrize("layout", ["padded_rows", "every_other_sequence"])
+def test_strided_cache_matches_contiguous_and_oracle(lib, layout):
+    # The cache as a view of a larger buffer (rows padded to 640 values, or every
+    # other sequence of a batch twice as large), NaN everywhere the view does not
+    # cover: the same output, bit for bit, as the contiguous cache.
+    cfg = _v3((300, 17, 129), 2)
+    P = Problem(lib, cfg)
+    ref_out = P.decode(opts=lib.opts(num_pairs=5)).clone()
+    T_max = P.cache.shape[1]
+    if layout == "padded_rows":
+        big = torch.full((cfg.B, T_max, 640), float("nan"), dtype=torch.bfloat16, device="cuda")
+        view = big[:, :, :cfg.row]
+    else:
+        big = torch.full((2 * cfg.B, T_max, cfg.row), float("nan"), dtype=torch.bfloat16, device="cuda")
+        view = big[::2]
+    view.copy_(P.cache)
+    out = lib.decode(P.dims, P.qn, P.qr, P.W_UK, P.W_UV, view, P.seqlens, opts=lib.opts(num_pairs=5))
+    assert lib.device_status() == 0
+    assert torch.equal(out, ref_out)
+    check_close(as_f64(out), P.oracle_expanded(range(cfg.B)), "bf16", f"cache layout {layout}")
+
+
 def test_repeat_runs_are_bitwise_equal(lib):
     cfg = _v3((900, 77), 2)
     P = Problem(lib, cfg)
