@@ -429,7 +429,8 @@ def time_projections(torch, lib, dims, cfg, device, attn_out, flush, steps):
 
 
 class OracleSample:
-    """The fp64 expanded oracle on this host, on a bounded sample of (sequence 0, heads)."""
+    """The fp64 expanded oracle on this host, on a bounded sample of (sequence 0, heads),
+    and beside it the fp64 absorbed CPU form (all heads of sequence 0)."""
 
     def __init__(self, cfg):
         self.cfg = cfg
@@ -462,7 +463,18 @@ class OracleSample:
         sample = (f"sequence 0 (T={cfg.seqlens[0]}) x {n_heads} of {cfg.H} heads x {cfg.q_len} query token(s), "
                   f"fp64 expanded K/V; per-step time extrapolated linearly in heads x history length")
         return {"value": round(full_s * 1e6, 1), "unit": "us/step", "cores": int(self.cores), "kind": "oracle",
-                "sample": sample, "sample_seconds": round(dt, 3)}
+                "sample": sample, "sample_seconds": round(dt, 3), "absorbed": self.measure_absorbed()}
+
+    def measure_absorbed(self):
+        from oracle import decode_absorbed
+        cfg = self.cfg
+        t0 = time.perf_counter()
+        decode_absorbed(*self.args, seqs=[0])
+        dt = time.perf_counter() - t0
+        return {"value": round(dt / cfg.seqlens[0] * sum(cfg.seqlens) * 1e6, 1), "unit": "us/step",
+                "sample": f"sequence 0 (T={cfg.seqlens[0]}) x all {cfg.H} heads x {cfg.q_len} query token(s), fp64 "
+                          f"absorbed CPU form; per-step time extrapolated linearly in history length",
+                "sample_seconds": round(dt, 3)}
 
 
 def cpu_baseline(cfg, budget_s):

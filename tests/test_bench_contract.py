@@ -29,6 +29,7 @@ def test_reference_arm_prints_one_contract_line():
     assert d["config"]["workload"].startswith("v3_ragged")
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
+    assert cb["absorbed"]["value"] > 0 and cb["absorbed"]["unit"] == "us/step" and cb["absorbed"]["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": "us/step", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
 
 
