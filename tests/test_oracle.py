@@ -164,6 +164,26 @@ def test_output_projection_folds_with_W_UV():
 
 # ------------------------------------------------------------------ decode: closed forms
 
+def test_softmax_hand_example_and_invariants():
+    # The softmax the decode applies per score row: weights proportional to
+    # e^s that sum to one, unchanged by a constant shift, and [0, ln 2] gives
+    # [1/3, 2/3] by hand.
+    from oracle.mla_oracle import _softmax
+
+    np.testing.assert_allclose(_softmax(np.array([0.0, math.log(2.0)])), [1.0 / 3.0, 2.0 / 3.0], rtol=1e-15)
+    rng = np.random.default_rng(8)
+    for n in (1, 7, 4096):
+        s = rng.standard_normal(n) * 10.0
+        p = _softmax(s)
+        assert abs(p.sum() - 1.0) < 1e-12 and (p >= 0).all()
+        np.testing.assert_allclose(_softmax(s + 123.25), p, rtol=1e-12, atol=1e-300)
+        np.testing.assert_allclose(p[1:] / p[:-1] if n > 1 else p, np.exp(np.diff(s)) if n > 1 else [1.0],
+                                   rtol=1e-9)
+    # a score of -inf (a key the query may not see) gets weight zero
+    p = _softmax(np.array([0.5, -np.inf, 0.5]))
+    np.testing.assert_array_equal(p, [0.5, 0.0, 0.5])
+
+
 def test_single_token_history_returns_W_UV_c():
     # T = 1: the softmax over one key is 1, so out_h = W_UV[h] c_0 whatever the query.
     qn, qr, W_UK, W_UV, hist = _rand_problem(np.random.default_rng(4), T=(1, 1))
